@@ -1,0 +1,191 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) DeepSeek-V3-style Mixture-of-Experts
+ * layer forward pass.
+ *
+ * The layer (pages "DeepSeek-V3.2-Exp - Expert scores" and "DeepSeek-V3.2-Exp
+ * - Weighted expert sum"; the MoE class on the hackaday page "time to jump
+ * right in and swim with the big fish"):
+ *
+ *   z      = x . W_r^T                        fp32 router logits   (moe_gate)
+ *   s      = sigmoid(z) | softmax(z)          unbiased scores
+ *   b      = s + bias                         selection-only bias
+ *   groups = top-topk_groups of n_groups contiguous expert blocks, scored by
+ *            the sum of their top-2 b (with a bias) or their max b (without)
+ *   idx    = top-k of b outside the dropped groups, descending b
+ *   w      = s[idx] (/ sum, for sigmoid) * route_scale
+ *   counts = bincount(idx), offsets = exclusive scan    (moe_dispatch)
+ *   E_e(x) = w2_e (silu(w1_e x) * (w3_e x))   SwiGLU     (moe_experts_grouped)
+ *   y[t]   = sum_j w[t,j] E_{idx[t,j]}(x[t]) + S(x[t])  (moe_combine)
+ *            accumulated in fp32, cast back to the activation dtype once.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major
+ *     and contiguous, 16-byte aligned. "act" means the activation dtype of the
+ *     config (fp32 or bf16): x, the router weight, all expert weights, the
+ *     intermediates and y use it. The selection bias and the routing weights
+ *     are always fp32; expert indices and all counts/offsets are int32.
+ *   - Weights are stored [out, in]: W_r [E, D], w1/w3 [E, I, D], w2 [E, D, I],
+ *     shared ws1/ws3 [I_s, D], ws2 [D, I_s] (I_s = shared_inter).
+ *   - The library allocates no device memory. Scratch comes from the caller's
+ *     workspace `ws` of at least moe_workspace_size() bytes, which must be
+ *     zeroed once by moe_workspace_init() after allocation. A workspace may be
+ *     reused by any sequence of calls on one stream; calls that share a
+ *     workspace must not run concurrently.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *     asynchronous on it and never synchronises the host, except
+ *     moe_check_error.
+ *   - Argument checks are synchronous: a bad config, size or pointer returns
+ *     MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE before
+ *     anything is launched. A failed launch returns MOE_ERR_CUDA.
+ *   - Conditions only the device can see (an expert index outside [0, E)
+ *     handed to moe_dispatch, a pipeline wait that exceeded its time limit)
+ *     set a sticky error word in the workspace; the offending element is
+ *     skipped, nothing is written out of bounds. moe_check_error() reads and
+ *     clears it.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad size or config */
+  MOE_ERR_UNSUPPORTED = -2,  /* a valid config this library does not run   */
+  MOE_ERR_WORKSPACE = -3,    /* workspace missing or smaller than required  */
+  MOE_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed         */
+  MOE_ERR_DEVICE_CHECK = -5, /* a device-side check failed (bad index)       */
+  MOE_ERR_TIMEOUT = -6       /* a device pipeline wait hit its time limit    */
+} moe_status;
+
+typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype;
+typedef enum { MOE_SCORE_SIGMOID = 0, MOE_SCORE_SOFTMAX = 1 } moe_score;
+
+/* Layer shape, mirroring the Gate/MoE constructor arguments on the pages:
+ * dim, n_routed_experts, n_expert_groups, n_limited_groups,
+ * n_activated_experts, moe_inter_dim, n_shared_experts * moe_inter_dim,
+ * score_func, route_scale, and whether the selection bias exists.
+ * Limits: 1 <= n_routed <= 1024; n_groups divides n_routed, n_groups <= 64 and
+ * the group width n_routed/n_groups is a power of two <= 32 or a multiple of
+ * 32; 1 <= topk_groups <= n_groups; 1 <= topk <= min(32, topk_groups *
+ * n_routed / n_groups); group width >= 2 when has_bias and n_groups > 1;
+ * dim, moe_inter, shared_inter multiples of 8 (bf16) / 4 (fp32);
+ * shared_inter may be 0 (no shared expert). */
+typedef struct {
+  int32_t dim;
+  int32_t n_routed;
+  int32_t n_groups;
+  int32_t topk_groups;
+  int32_t topk;
+  int32_t moe_inter;
+  int32_t shared_inter;
+  int32_t score;       /* moe_score */
+  float route_scale;
+  int32_t has_bias;    /* 0 or 1 */
+  int32_t dtype;       /* moe_dtype */
+} moe_config;
+
+/* Bytes of workspace every call below needs for T tokens (T >= 1). */
+MOE_API moe_status moe_workspace_size(const moe_config* cfg, int64_t T, size_t* bytes);
+
+/* Zero the workspace header (the sticky error word). Call once after
+ * allocating the workspace, before any other call that uses it. */
+MOE_API moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Router (page "Expert scores", Gate.forward): fp32 logits from x [T, D] (act)
+ * and W_r [E, D] (act), scores, bias (fp32 [E], ignored unless has_bias;
+ * may be NULL only then), group limit, top-k.
+ * Out: weights [T, k] fp32 and idx [T, k] int32, each token's picks ordered
+ * by descending biased score, ties to the lower expert index. */
+MOE_API moe_status moe_gate(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                    const float* bias, float* weights, int32_t* idx,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch (page "Weighted expert sum": bincount, then each expert's rows in
+ * row-major order of idx): counts [E], offsets [E+1] (exclusive scan,
+ * offsets[E] = number of valid pairs), src [T*k] (token of each permuted
+ * row), pos [T*k] (permuted row of pair (t, j), -1 for an invalid index), and
+ * x_perm [T*k, D] (act), x's rows in expert-contiguous order, ascending token
+ * within an expert. An index outside [0, E) sets MOE_ERR_DEVICE_CHECK in the
+ * error word and its pair is dropped. */
+MOE_API moe_status moe_dispatch(const moe_config* cfg, int64_t T, const int32_t* idx, const void* x,
+                        int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
+                        void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Experts (each Expert(dim, moe_inter_dim) and the shared MLP of width
+ * n_shared_experts * moe_inter_dim; SwiGLU body): for every expert e, rows
+ * [offsets[e], offsets[e+1]) of x_perm [T*k, D] go through expert e into
+ * y_perm [T*k, D] (act); x [T, D] goes through the shared MLP into s [T, D]
+ * (act). h = silu(w1 x) * (w3 x) is formed in fp32 and rounded to act before
+ * w2. x, ws1, ws3, ws2 and s may be NULL when shared_inter == 0. Rows of
+ * y_perm at or past offsets[E] are not written. */
+MOE_API moe_status moe_experts_grouped(const moe_config* cfg, int64_t T, const void* x_perm,
+                               const int32_t* offsets, const void* w1, const void* w3,
+                               const void* w2, const void* x, const void* ws1,
+                               const void* ws3, const void* ws2, void* y_perm, void* s,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* Combine (page "Weighted expert sum": y_routed = sum_i G_i E_i, accumulated
+ * in float32 and cast back at the end; then the shared expert added):
+ * y[t] = act( sum_j weights[t,j] * y_perm[pos[t,j]] + s[t] ), fp32 sum over
+ * j = 0..k-1 then s. Pairs with pos < 0 are skipped; s may be NULL. */
+MOE_API moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_perm,
+                       const int32_t* pos, const float* weights, const void* s, void* y,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer (MoE.forward): gate, dispatch, experts and combine chained
+ * on `stream` with no host synchronisation. y [T, D] (act). weights_out
+ * [T, k] and idx_out [T, k] may be NULL; when given they receive the routing. */
+MOE_API moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                       const float* bias, const void* w1, const void* w3, const void* w2,
+                       const void* ws1, const void* ws3, const void* ws2, void* y,
+                       float* weights_out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Synchronise `stream`, read and clear the workspace's error word. Returns
+ * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT (or MOE_ERR_CUDA). */
+MOE_API moe_status moe_check_error(void* ws, void* stream);
+
+/* Static text for a status code. */
+MOE_API const char* moe_status_string(moe_status st);
+
+/* Number of kernels moe_forward launches for this config (for accounting). */
+MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
+
+/* Per-kernel timing of moe_forward, for measurement (off by default).
+ * moe_stage_timing_begin(max_calls) creates max_calls * 9 CUDA events (no
+ * device memory) and arms the next max_calls moe_forward calls to record one
+ * event on their stream before their first kernel and one after each of their
+ * moe_forward_launch_count() kernels. moe_stage_timing_end(ms, n) disarms,
+ * waits for the recorded events and writes to ms[i] the total milliseconds
+ * kernel i (launch order: router logits, router select, dispatch rank,
+ * dispatch scan, dispatch scatter, experts up, experts down, combine) took
+ * over the recorded calls, for i < n <= 8; it returns the number of calls
+ * recorded, or a negative moe_status. Single-threaded use only. */
+MOE_API moe_status moe_stage_timing_begin(int32_t max_calls);
+MOE_API int32_t moe_stage_timing_end(float* ms, int32_t n);
+
+/* Which kernel runs the expert GEMMs of a bf16 layer, process-wide:
+ * AUTO (default) and TCGEN05 use the tensor-core grouped GEMM; SIMT uses the
+ * CUDA-core grouped GEMM that fp32 layers always use. SIMT is a slow
+ * independent cross-check of the tensor-core kernel, not a fallback: nothing
+ * switches to it on its own. Returns MOE_ERR_INVALID_ARG for other values. */
+enum { MOE_EXPERT_KERNEL_AUTO = 0, MOE_EXPERT_KERNEL_SIMT = 1, MOE_EXPERT_KERNEL_TCGEN05 = 2 };
+MOE_API moe_status moe_select_expert_kernel(int32_t which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

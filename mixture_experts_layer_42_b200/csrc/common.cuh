@@ -1,0 +1,192 @@
+// Internal helpers shared by the kernels of the MoE layer library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// Bits of the sticky device error word (first 4 bytes of the workspace).
+enum : uint32_t {
+  ERRBIT_BAD_INDEX = 1u,   // an expert index outside [0, E)
+  ERRBIT_TIMEOUT = 2u,     // a pipeline wait hit its time limit
+};
+
+// Alignment of every workspace region (bytes).
+constexpr size_t kWsAlign = 256;
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+template <typename T>
+__host__ __device__ inline T ceil_div(T a, T b) { return (a + b - 1) / b; }
+
+// Tokens per dispatch chunk (the unit of the stable counting sort).
+constexpr int kDispatchChunkTokens = 64;
+
+// Router GEMM tile: 128 tokens x 64 experts, 32-deep k slices.
+constexpr int kRouterBM = 128;
+constexpr int kRouterBN = 64;
+constexpr int kRouterBK = 32;
+
+struct WsLayout {
+  size_t header;        // error word
+  size_t router_part;   // [splits, T, E] fp32
+  size_t chunk_hist;    // [n_chunks, E] int32
+  size_t pos_local;     // [T * k] int32, ranks within a dispatch chunk
+  size_t weights;       // [T, k] fp32
+  size_t idx;           // [T, k] int32
+  size_t counts;        // [E] int32
+  size_t offsets;       // [E + 1] int32
+  size_t src;           // [T * k] int32
+  size_t pos;           // [T * k] int32
+  size_t x_perm;        // [T * k, D] act
+  size_t y_perm;        // [T * k, D] act
+  size_t s;             // [T, D] act
+  size_t h;             // [T * k, I] act
+  size_t hs;            // [T, I_s] act
+  size_t total;
+  int router_splits;
+  int n_chunks;
+};
+
+inline int act_bytes(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
+
+// CTAs the router GEMM aims for (two per SM of a 148-SM B200).
+constexpr int kRouterTargetCtas = 296;
+
+// Number of k splits of the router GEMM for T tokens: enough CTAs to reach
+// the target, at most 32 splits, each split at least 4 k slices deep. Depends
+// only on the shape, so the workspace size is a pure function of it.
+inline int router_splits(const moe_config& c, int64_t T) {
+  int64_t tiles = ceil_div<int64_t>(T, kRouterBM) * ceil_div<int64_t>(c.n_routed, kRouterBN);
+  int64_t want = (kRouterTargetCtas + tiles - 1) / tiles;
+  int64_t kslices = ceil_div<int64_t>(c.dim, kRouterBK);
+  int64_t maxs = kslices / 4 > 0 ? kslices / 4 : 1;
+  if (want > 32) want = 32;
+  if (want > maxs) want = maxs;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+inline WsLayout ws_layout(const moe_config& c, int64_t T) {
+  WsLayout L{};
+  const int64_t E = c.n_routed, k = c.topk, D = c.dim, I = c.moe_inter, Is = c.shared_inter;
+  const int64_t ab = act_bytes(c);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + (bytes ? bytes : 1), kWsAlign);
+    return o;
+  };
+  L.router_splits = router_splits(c, T);
+  L.n_chunks = (int)ceil_div<int64_t>(T, kDispatchChunkTokens);
+  L.header = take(kWsAlign);
+  L.router_part = take((size_t)L.router_splits * T * E * 4);
+  L.chunk_hist = take((size_t)L.n_chunks * E * 4);
+  L.pos_local = take((size_t)T * k * 4);
+  L.weights = take((size_t)T * k * 4);
+  L.idx = take((size_t)T * k * 4);
+  L.counts = take((size_t)E * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.src = take((size_t)T * k * 4);
+  L.pos = take((size_t)T * k * 4);
+  L.x_perm = take((size_t)T * k * D * ab);
+  L.y_perm = take((size_t)T * k * D * ab);
+  L.s = take((size_t)T * D * ab);
+  L.h = take((size_t)T * k * I * ab);
+  L.hs = take((size_t)T * (Is > 0 ? Is : 1) * ab);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- device
+
+__device__ __forceinline__ void set_error(uint32_t* err, uint32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// 16-byte vector of activations: 8 bf16 or 4 fp32.
+template <typename T> struct Vec16;
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  uint4 raw;
+  __device__ __forceinline__ void to_float(float* f) const {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 t = __bfloat1622float2(p[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+  __device__ __forceinline__ void from_float(const float* f) {
+    __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  }
+};
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  uint4 raw;
+  __device__ __forceinline__ void to_float(float* f) const {
+    f[0] = __uint_as_float(raw.x);
+    f[1] = __uint_as_float(raw.y);
+    f[2] = __uint_as_float(raw.z);
+    f[3] = __uint_as_float(raw.w);
+  }
+  __device__ __forceinline__ void from_float(const float* f) {
+    raw = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                     __float_as_uint(f[3]));
+  }
+};
+
+// ---------------------------------------------------------------- launchers
+
+// Operands of one grouped expert launch ([0] routed experts, [1] shared MLP).
+struct GroupedArgs {
+  const void* a[2];     // A rows: [0] x_perm / h, [1] x / hs
+  const void* b1[2];    // w1 / w2 stacked [E, N, K]; shared ws1 / ws2 [N_s, K_s]
+  const void* b3[2];    // w3 / ws3 (UP only)
+  void* out[2];         // [0] h / y_perm, [1] hs / s
+  int n[2];             // output columns per group kind
+  int kdim[2];          // reduction depth per group kind
+  const int32_t* offsets;
+  int E;
+  int64_t t_shared;     // rows of the shared group (0: none)
+};
+
+// Records the next per-kernel timing event on `st` when moe_forward runs with
+// stage timing on (see moe_stage_timing_begin); a no-op otherwise. Every
+// launcher calls it right after each kernel it launches.
+void stage_mark(cudaStream_t st);
+
+cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
+                          const float* bias, float* weights, int32_t* idx, float* part,
+                          int splits, cudaStream_t st);
+cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
+                            int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
+                            void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,
+                            uint32_t* err, cudaStream_t st);
+cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, const int32_t* pos,
+                           const float* weights, const void* s, void* y, cudaStream_t st);
+cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
+                                cudaStream_t st);
+cudaError_t launch_grouped_tc(bool up, int64_t Tk, int64_t T_sh, int E, const void* a0,
+                              const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
+                              const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
+                              void* out1, const int32_t* offsets, uint32_t* err, int num_sms,
+                              cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,371 @@
+// C ABI of the MoE layer library: argument checks, workspace carving and the
+// launch sequence of each entry point (declared in include/moe.h).
+#include "common.cuh"
+
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+namespace moe {
+
+namespace {
+
+// Which kernel runs the expert GEMMs of a bf16 layer (see moe_select_expert_kernel).
+int g_expert_kernel = MOE_EXPERT_KERNEL_AUTO;
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+moe_status check_config(const moe_config* c, int64_t T) {
+  if (!c || T < 1) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_DT_F32 && c->dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->score != MOE_SCORE_SIGMOID && c->score != MOE_SCORE_SOFTMAX) return MOE_ERR_INVALID_ARG;
+  if (c->has_bias != 0 && c->has_bias != 1) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(c->route_scale)) return MOE_ERR_INVALID_ARG;
+  const int E = c->n_routed, G = c->n_groups;
+  if (E < 1 || G < 1 || c->topk < 1 || c->topk_groups < 1) return MOE_ERR_INVALID_ARG;
+  if (E % G != 0 || c->topk_groups > G) return MOE_ERR_INVALID_ARG;
+  const int per = E / G;
+  if (c->topk > c->topk_groups * per) return MOE_ERR_INVALID_ARG;   // -inf never picked
+  if (c->has_bias && G > 1 && per < 2) return MOE_ERR_INVALID_ARG;  // top-2 group score
+  if (c->dim < 1 || c->moe_inter < 1 || c->shared_inter < 0) return MOE_ERR_INVALID_ARG;
+  const int q = c->dtype == MOE_DT_BF16 ? 8 : 4;  // 16-byte rows
+  if (c->dim % q || c->moe_inter % q || c->shared_inter % q) return MOE_ERR_INVALID_ARG;
+  if (E > 1024 || G > 64 || c->topk > 32) return MOE_ERR_UNSUPPORTED;
+  if (G > 1 && !((per <= 32 && is_pow2(per)) || per % 32 == 0)) return MOE_ERR_UNSUPPORTED;
+  if (T * c->topk > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config& c, int64_t T, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = ws_layout(c, T);
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < L->total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
+}
+
+int num_sms_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Make this thread's current device the one the caller's work lives on: the
+// stream's device, or for the legacy default stream the device of `ptr`.
+// The library carries its own copy of the CUDA runtime, whose current device
+// does not follow the caller's runtime.
+moe_status bind_device(cudaStream_t s, const void* ptr) {
+  int dev = -1;
+  if (s) {
+    if (cudaStreamGetDevice(s, &dev) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, ptr) != cudaSuccess) return MOE_ERR_INVALID_ARG;
+    if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
+      return MOE_ERR_INVALID_ARG;
+    dev = pa.device;
+  }
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cur != dev && cudaSetDevice(dev) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* offsets,
+                       const void* w1, const void* w3, const void* w2, const void* x,
+                       const void* ws1, const void* ws3, const void* ws2, void* y_perm, void* s,
+                       void* h, void* hs, uint32_t* err, cudaStream_t st) {
+  const int64_t Tk = T * c.topk;
+  const bool sh = c.shared_inter > 0;
+  const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
+  if (tc) {
+    cudaError_t e = launch_grouped_tc(true, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
+                                      c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
+                                      err, num_sms_current(), st);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_grouped_tc(false, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
+                          c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, err,
+                          num_sms_current(), st);
+    return cuda_status(e);
+  }
+  GroupedArgs g;
+  memset(&g, 0, sizeof(g));
+  g.offsets = offsets;
+  g.E = c.n_routed;
+  g.t_shared = sh ? T : 0;
+  g.a[0] = x_perm; g.a[1] = x;
+  g.b1[0] = w1; g.b1[1] = ws1;
+  g.b3[0] = w3; g.b3[1] = ws3;
+  g.out[0] = h; g.out[1] = hs;
+  g.n[0] = c.moe_inter; g.n[1] = c.shared_inter;
+  g.kdim[0] = c.dim; g.kdim[1] = c.dim;
+  cudaError_t e = launch_grouped_simt(c, T, true, g, st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  g.a[0] = h; g.a[1] = hs;
+  g.b1[0] = w2; g.b1[1] = ws2;
+  g.b3[0] = nullptr; g.b3[1] = nullptr;
+  g.out[0] = y_perm; g.out[1] = s;
+  g.n[0] = c.dim; g.n[1] = c.dim;
+  g.kdim[0] = c.moe_inter; g.kdim[1] = c.shared_inter;
+  return cuda_status(launch_grouped_simt(c, T, false, g, st));
+}
+
+// Per-kernel timing of moe_forward (moe_stage_timing_begin / _end).
+struct StageTiming {
+  bool on = false;        // armed by moe_stage_timing_begin
+  bool in_forward = false;
+  int max_calls = 0;
+  int calls = 0;          // moe_forward calls recorded
+  int marks = 0;          // events recorded in the current call
+  int per_call = 0;       // events per call (kernels + 1)
+  std::vector<cudaEvent_t> ev;
+};
+StageTiming g_timing;
+
+}  // namespace
+
+void stage_mark(cudaStream_t st) {
+  StageTiming& T = g_timing;
+  if (!T.on || !T.in_forward || T.marks >= T.per_call) return;
+  cudaEventRecord(T.ev[(size_t)T.calls * T.per_call + T.marks], st);
+  ++T.marks;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_config* cfg, int64_t T, size_t* bytes) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = ws_layout(*cfg, T).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsAlign || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  moe_status st = bind_device((cudaStream_t)stream, ws);
+  if (st != MOE_OK) return st;
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsAlign, (cudaStream_t)stream));
+}
+
+moe_status moe_gate(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                    const float* bias, float* weights, int32_t* idx, void* ws, size_t ws_bytes,
+                    void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(weights) || !aligned16(idx))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->has_bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
+  return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx,
+                                   at<float>(ws, L.router_part), L.router_splits,
+                                   (cudaStream_t)stream));
+}
+
+moe_status moe_dispatch(const moe_config* cfg, int64_t T, const int32_t* idx, const void* x,
+                        int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
+                        void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(idx) || !aligned16(x) || !aligned16(counts) || !aligned16(offsets) ||
+      !aligned16(src) || !aligned16(pos) || !aligned16(x_perm))
+    return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
+  return cuda_status(launch_dispatch(*cfg, T, idx, x, counts, offsets, src, pos, x_perm,
+                                     at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local),
+                                     L.n_chunks, at<uint32_t>(ws, L.header), (cudaStream_t)stream));
+}
+
+moe_status moe_experts_grouped(const moe_config* cfg, int64_t T, const void* x_perm,
+                               const int32_t* offsets, const void* w1, const void* w3,
+                               const void* w2, const void* x, const void* ws1, const void* ws3,
+                               const void* ws2, void* y_perm, void* s, void* ws, size_t ws_bytes,
+                               void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(x_perm) || !aligned16(offsets) || !aligned16(w1) || !aligned16(w3) ||
+      !aligned16(w2) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->shared_inter > 0 && (!aligned16(x) || !aligned16(ws1) || !aligned16(ws3) ||
+                                !aligned16(ws2) || !aligned16(s)))
+    return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
+  return run_experts(*cfg, T, x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, y_perm, s,
+                     at<void>(ws, L.h), at<void>(ws, L.hs), at<uint32_t>(ws, L.header),
+                     (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const int32_t* pos,
+                       const float* weights, const void* s, void* y, void* ws, size_t ws_bytes,
+                       void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(y_perm) || !aligned16(pos) || !aligned16(weights) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  if (s && !aligned16(s)) return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
+  return cuda_status(launch_combine(*cfg, T, y_perm, pos, weights, s, y, (cudaStream_t)stream));
+}
+
+moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                       const float* bias, const void* w1, const void* w3, const void* w2,
+                       const void* ws1, const void* ws3, const void* ws2, void* y,
+                       float* weights_out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(w3) ||
+      !aligned16(w2) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  if (c.has_bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0 && (!aligned16(ws1) || !aligned16(ws3) || !aligned16(ws2)))
+    return MOE_ERR_INVALID_ARG;
+  if ((weights_out && !aligned16(weights_out)) || (idx_out && !aligned16(idx_out)))
+    return MOE_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((st = check_ws(c, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = bind_device(s, ws)) != MOE_OK) return st;
+  StageTiming& TM = g_timing;
+  TM.in_forward = TM.on && TM.calls < TM.max_calls;
+  if (TM.in_forward) {
+    TM.marks = 0;
+    stage_mark(s);
+  }
+  struct EndCall {
+    StageTiming& t;
+    ~EndCall() {
+      if (t.in_forward) {
+        if (t.marks == t.per_call) ++t.calls;
+        t.in_forward = false;
+      }
+    }
+  } end_call{TM};
+  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+  uint32_t* err = at<uint32_t>(ws, L.header);
+  if (launch_router(c, T, x, w_router, bias, weights, idx, at<float>(ws, L.router_part),
+                    L.router_splits, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* pos = at<int32_t>(ws, L.pos);
+  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, at<int32_t>(ws, L.src),
+                      pos, at<void>(ws, L.x_perm), at<int32_t>(ws, L.chunk_hist),
+                      at<int32_t>(ws, L.pos_local), L.n_chunks, err, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const bool sh = c.shared_inter > 0;
+  void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
+  st = run_experts(c, T, at<void>(ws, L.x_perm), offsets, w1, w3, w2, x, ws1, ws3, ws2,
+                   at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs), err, s);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
+}
+
+moe_status moe_check_error(void* ws, void* stream) {
+  if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  moe_status st = bind_device(s, ws);
+  if (st != MOE_OK) return st;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & ERRBIT_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (word & ERRBIT_BAD_INDEX) return MOE_ERR_DEVICE_CHECK;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "device-side check failed (expert index out of range)";
+    case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
+  if (check_config(cfg, T) != MOE_OK) return -1;
+  // router: logits + select; dispatch: rank + scan + scatter; experts: up +
+  // down; combine
+  return 2 + 3 + 2 + 1;
+}
+
+moe_status moe_stage_timing_begin(int32_t max_calls) {
+  StageTiming& T = g_timing;
+  if (max_calls < 1 || max_calls > 4096) return MOE_ERR_INVALID_ARG;
+  for (cudaEvent_t e : T.ev) cudaEventDestroy(e);
+  T.ev.clear();
+  T.per_call = 2 + 3 + 2 + 1 + 1;
+  T.ev.resize((size_t)max_calls * T.per_call, nullptr);
+  for (auto& e : T.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
+  T.max_calls = max_calls;
+  T.calls = 0;
+  T.on = true;
+  return MOE_OK;
+}
+
+int32_t moe_stage_timing_end(float* ms, int32_t n) {
+  StageTiming& T = g_timing;
+  if (!T.on) return MOE_ERR_INVALID_ARG;
+  T.on = false;
+  const int kernels = T.per_call - 1;
+  if (!ms || n < 1 || n > kernels) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) ms[i] = 0.f;
+  for (int c = 0; c < T.calls; ++c) {
+    for (int i = 0; i < n; ++i) {
+      cudaEvent_t a = T.ev[(size_t)c * T.per_call + i], b = T.ev[(size_t)c * T.per_call + i + 1];
+      if (cudaEventSynchronize(b) != cudaSuccess) return MOE_ERR_CUDA;
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, a, b) != cudaSuccess) return MOE_ERR_CUDA;
+      ms[i] += t;
+    }
+  }
+  return T.calls;
+}
+
+moe_status moe_select_expert_kernel(int32_t which) {
+  if (which != MOE_EXPERT_KERNEL_AUTO && which != MOE_EXPERT_KERNEL_SIMT &&
+      which != MOE_EXPERT_KERNEL_TCGEN05)
+    return MOE_ERR_INVALID_ARG;
+  g_expert_kernel = which;
+  return MOE_OK;
+}
+
+}  // extern "C"
