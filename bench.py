@@ -61,7 +61,20 @@ def parse():
     ap.add_argument("--cpu-tokens", type=int, default=0,
                     help="tokens in the CPU oracle sample (0: sized to ~15 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T of the workload (smaller cases for profiling)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the number of routed experts (smaller cases for profiling)")
     return ap.parse_args()
+
+
+def workload(a):
+    cfg = inputs.CONFIGS[a.config]
+    if a.tokens:
+        cfg = cfg.with_(T=a.tokens, name=f"{cfg.name}[T={a.tokens}]")
+    if a.experts:
+        cfg = cfg.with_(n_routed=a.experts, name=f"{cfg.name}[E={a.experts}]")
+    return cfg
 
 
 # ---------------------------------------------------------------- distributed
@@ -112,7 +125,7 @@ def peaks():
 class Clocks:
     """nvidia-smi samples of the SM clock and throttle reasons, every 100 ms."""
 
-    Q = ("timestamp,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -124,7 +137,7 @@ class Clocks:
         except OSError:
             self.p = None
 
-    def stop(self, t0, t1, bus_id):
+    def stop(self, t0, t1, uuid):
         if self.p is None:
             return None
         self.p.terminate()
@@ -145,7 +158,7 @@ class Clocks:
             except ValueError:
                 continue
         os.unlink(self.f.name)
-        mine = [r for r in rows if bus_id and bus_id.lower()[-12:] in r[1]] or rows
+        mine = [r for r in rows if uuid and uuid.lower() in r[1]] or rows
         inside = [r for r in mine if t0 <= r[0] <= t1]
         window = "timed"
         if len(inside) < 3:
@@ -153,7 +166,7 @@ class Clocks:
         if not inside:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[5][1:5]) if "Active" in v})
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[5][1:5]) if v.strip() == "Active"})
         return {"sm_mhz": float(np.median([r[2] for r in inside])), "sm_max_mhz": max(r[3] for r in inside),
                 "reasons": reasons, "samples": len(inside), "window": window,
                 "power_w_max": max(r[4] for r in inside)}
@@ -253,7 +266,7 @@ def reference_arm(a, D):
     """The CPU oracle, as it stands, on the host cores (rank 0 only)."""
     if D.rank != 0:
         return
-    cfg = inputs.CONFIGS[a.config]
+    cfg = workload(a)
     x, w_r, bias = inputs.routing_inputs(cfg)
     w = inputs.expert_weights(cfg, "cuda" if torch.cuda.is_available() else "cpu")
     n_tok = a.cpu_tokens or (8 if cfg.dim >= 4096 else 64)
@@ -278,7 +291,7 @@ def reference_arm(a, D):
 
 def ours_arm(a, D):
     from mixture_experts_layer_42_b200 import binding as M
-    cfg = inputs.CONFIGS[a.config]
+    cfg = workload(a)
     dev = torch.device("cuda", torch.cuda.current_device())
     x_cpu, w_r_cpu, bias_cpu = inputs.routing_inputs(cfg)
     x = x_cpu.to(dev)
@@ -303,9 +316,9 @@ def ours_arm(a, D):
         raise RuntimeError("device error word set after the first forward")
     n_active = int((torch.bincount(idx.flatten().long(), minlength=cfg.n_routed) > 0).sum().item())
 
-    bus = None
+    uuid = None
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except AttributeError:
         pass
     clocks = Clocks() if D.rank == 0 else None
@@ -358,7 +371,7 @@ def ours_arm(a, D):
     D.barrier()
     torch.cuda.synchronize()
     ms_e2e = D.max(e0.elapsed_time(e1))
-    ck = clocks.stop(wall0, wall1, bus) if clocks else None
+    ck = clocks.stop(wall0, wall1, uuid) if clocks else None
 
     N = D.world
     value = N * T * a.steps / (ms / 1e3)

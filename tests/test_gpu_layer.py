@@ -105,7 +105,7 @@ def test_gate_softmax_ties_lowest_index():
     ws = M.alloc_workspace(cfg, L.T)
     M.moe_gate(cfg, L.x, L.w_r, None, wts, idx, ws)
     assert (idx.cpu() == torch.arange(6, dtype=torch.int32)).all()
-    np.testing.assert_allclose(wts.cpu().numpy(), 1.0 / 64, rtol=1e-6)
+    np.testing.assert_allclose(wts.cpu().numpy(), cfg.route_scale / 64, rtol=1e-6)
 
 
 # ---------------------------------------------------------------- dispatch
