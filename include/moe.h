@@ -163,6 +163,26 @@ MOE_API const char* moe_status_string(moe_status st);
 /* Number of kernels moe_forward launches for this config (for accounting). */
 MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
 
+/* moe_gate without a workspace. The pages have no counterpart of this call:
+ * it exists for callers that cannot allocate device memory or hand out a
+ * workspace -- for instance a plugin inside a host framework that owns every
+ * byte of device memory through its own pool, or a latency-critical serving
+ * loop where cudaMalloc is off limits because it can synchronise the device.
+ * Same arguments and results as moe_gate, minus ws / ws_bytes: the router's
+ * split-k partial sums go to a 4 MiB scratch array built into the library
+ * (1,048,576 floats; every GPU that loads the library holds it until the
+ * process exits). Limit: T * n_routed <= 1,048,576 (T <= 4096 at 256
+ * experts); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing. The
+ * call allocates no device memory. The first call on each device looks up the
+ * scratch's device address (cudaGetSymbolAddress) and caches it. All calls
+ * share the one array and it keeps the last call's partial sums (each call
+ * overwrites every element it reads); calls whose work overlaps on the GPU,
+ * on different streams or host threads, race on it and must be serialised
+ * by the caller. */
+MOE_API moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x,
+                                    const void* w_router, const float* bias, float* weights,
+                                    int32_t* idx, void* stream);
+
 /* Per-kernel timing of moe_forward, for measurement (off by default).
  * moe_stage_timing_begin(max_calls) creates max_calls * 9 CUDA events (no
  * device memory) and arms the next max_calls moe_forward calls to record one

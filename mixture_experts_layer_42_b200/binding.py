@@ -34,7 +34,7 @@ MOE_EXPERT_KERNEL_AUTO, MOE_EXPERT_KERNEL_SIMT, MOE_EXPERT_KERNEL_TCGEN05 = 0, 1
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch",
            "moe_experts_grouped", "moe_combine", "moe_forward", "moe_check_error",
            "moe_status_string", "moe_forward_launch_count", "moe_select_expert_kernel",
-           "moe_stage_timing_begin", "moe_stage_timing_end")
+           "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc")
 
 # Kernels of moe_forward, in launch order.
 STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_scatter",
@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "moe_select_expert_kernel": [I32],
         "moe_stage_timing_begin": [I32],
         "moe_stage_timing_end": [ctypes.POINTER(ctypes.c_float), I32],
+        "moe_gate_noalloc": [C, I64, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +147,12 @@ def alloc_workspace(cfg, T: int, device="cuda") -> torch.Tensor:
 def moe_gate(cfg, x, w_router, bias, weights, idx, ws, stream=None) -> None:
     _check(_lib.moe_gate(_c(cfg), x.shape[0], _p(x), _p(w_router), _p(bias), _p(weights), _p(idx),
                          _p(ws), ws.numel(), _s(stream)), "moe_gate")
+
+
+def moe_gate_noalloc(cfg, x, w_router, bias, weights, idx, stream=None) -> None:
+    """moe_gate with the library's built-in scratch instead of a workspace."""
+    _check(_lib.moe_gate_noalloc(_c(cfg), x.shape[0], _p(x), _p(w_router), _p(bias), _p(weights),
+                                 _p(idx), _s(stream)), "moe_gate_noalloc")
 
 
 def moe_dispatch(cfg, idx, x, counts, offsets, src, pos, x_perm, ws, stream=None) -> None:

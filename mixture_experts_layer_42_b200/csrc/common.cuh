@@ -175,6 +175,11 @@ void stage_mark(cudaStream_t st);
 cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
                           const float* bias, float* weights, int32_t* idx, float* part,
                           int splits, cudaStream_t st);
+// Built-in router scratch (moe_gate_noalloc): its size in floats, and its
+// device address on the current device.
+size_t gate_scratch_floats();
+cudaError_t gate_scratch_current_device(float** out);
+
 cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
                             int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                             void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,

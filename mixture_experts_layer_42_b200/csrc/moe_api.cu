@@ -326,6 +326,25 @@ int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
   return 2 + 3 + 2 + 1;
 }
 
+moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                            const float* bias, float* weights, int32_t* idx, void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(weights) || !aligned16(idx))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->has_bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  const int64_t per_split = T * (int64_t)cfg->n_routed;  // floats of one split's partials
+  if (per_split > (int64_t)gate_scratch_floats()) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = bind_device(s, x)) != MOE_OK) return st;
+  float* scratch = nullptr;
+  if (gate_scratch_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  int splits = router_splits(*cfg, T);
+  const int64_t fit = (int64_t)gate_scratch_floats() / per_split;
+  if (splits > fit) splits = (int)fit;
+  return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx, scratch, splits, s));
+}
+
 moe_status moe_stage_timing_begin(int32_t max_calls) {
   StageTiming& T = g_timing;
   if (max_calls < 1 || max_calls > 4096) return MOE_ERR_INVALID_ARG;

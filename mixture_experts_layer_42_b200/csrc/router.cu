@@ -17,6 +17,8 @@
 
 #include <float.h>
 
+#include <mutex>
+
 namespace moe {
 
 namespace {
@@ -357,6 +359,44 @@ cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const v
   else router_select_kernel<32><<<blocks, 256, 0, st>>>(a);
   stage_mark(st);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- built-in scratch
+//
+// moe_gate_noalloc runs the router with its split-k partial sums in this
+// file-scope device array instead of a caller workspace, for callers that
+// cannot allocate device memory. Every GPU that loads the library holds it
+// (4 MiB) until the process exits. Host code must not pass `g_gate_scratch`
+// itself to a kernel: on the host that name is only a stand-in; the device
+// address comes from cudaGetSymbolAddress, taken once per device.
+
+namespace {
+constexpr size_t kGateScratchFloats = size_t(1) << 20;
+static __device__ __align__(256) float g_gate_scratch[kGateScratchFloats];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_gate_scratch_mu;
+float* g_gate_scratch_addr[kMaxDevices] = {};
+}  // namespace
+
+size_t gate_scratch_floats() { return kGateScratchFloats; }
+
+// Device address of the built-in scratch on the current device; looked up on
+// the first call for each device (with that device current) and cached.
+cudaError_t gate_scratch_current_device(float** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_gate_scratch_mu);
+  if (!g_gate_scratch_addr[dev]) {
+    float* ptr = nullptr;
+    e = cudaGetSymbolAddress((void**)&ptr, g_gate_scratch);
+    if (e != cudaSuccess) return e;
+    g_gate_scratch_addr[dev] = ptr;
+  }
+  *out = g_gate_scratch_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace moe
