@@ -65,6 +65,8 @@ def parse():
                     help="override T of the workload (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the number of routed experts (smaller cases for profiling)")
+    ap.add_argument("--expert-kernel", default="auto", choices=["auto", "simt", "one_cta", "pair"],
+                    help="GEMM kernels of a bf16 layer (moe_select_expert_kernel)")
     return ap.parse_args()
 
 
@@ -305,6 +307,9 @@ def ours_arm(a, D):
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
     launches = M.moe_forward_launch_count(cfg, T)
+    M.moe_select_expert_kernel({"auto": M.MOE_EXPERT_KERNEL_AUTO, "simt": M.MOE_EXPERT_KERNEL_SIMT,
+                                "one_cta": M.MOE_EXPERT_KERNEL_TCGEN05,
+                                "pair": M.MOE_EXPERT_KERNEL_TCGEN05_PAIR}[a.expert_kernel])
 
     def step(xin=x, idx_out=None):
         M.moe_forward(cfg, xin, w_r, bias, *w, y, ws, idx_out=idx_out, stream=stream)
@@ -346,31 +351,62 @@ def ours_arm(a, D):
         raise RuntimeError("device error word set during the timed loop")
 
     # ------------------------------------------------------------ end to end (host buffers)
+    # Each step copies its x in from pinned host memory and its y back out.
+    # A serving loop overlaps them: the H2D of step i+1 (copy stream) and the
+    # D2H of step i (a second copy stream) run under the compute of the
+    # neighbouring steps, with double-buffered device x and y.
     x_h = x_cpu.pin_memory()
-    y_h = torch.empty(T, cfg.dim, dtype=cfg.torch_dtype).pin_memory()
-    x_dev = torch.empty_like(x)
+    y_h = [torch.empty(T, cfg.dim, dtype=cfg.torch_dtype).pin_memory() for _ in range(2)]
+    x_d = [torch.empty_like(x) for _ in range(2)]
+    y_d = [torch.empty_like(y) for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-    def e2e_step():
-        x_dev.copy_(x_h, non_blocking=True)
-        step(xin=x_dev)
-        y_h.copy_(y, non_blocking=True)
+    def e2e_run(n):
+        ev = lambda: torch.cuda.Event()
+        x_ready = [ev(), ev()]
+        done = [ev(), ev()]       # compute of the step that used buffer b
+        y_out = [ev(), ev()]      # D2H of buffer b finished
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        h2d.wait_event(start)
+        with torch.cuda.stream(h2d):
+            x_d[0].copy_(x_h, non_blocking=True)
+            x_ready[0].record(h2d)
+        for i in range(n):
+            b = i & 1
+            stream.wait_event(x_ready[b])
+            if i >= 2:
+                stream.wait_event(y_out[b])
+            M.moe_forward(cfg, x_d[b], w_r, bias, *w, y_d[b], ws, stream=stream)
+            done[b].record(stream)
+            if i + 1 < n:
+                nb = (i + 1) & 1
+                if i >= 1:
+                    h2d.wait_event(done[nb])
+                with torch.cuda.stream(h2d):
+                    x_d[nb].copy_(x_h, non_blocking=True)
+                    x_ready[nb].record(h2d)
+            d2h.wait_event(done[b])
+            with torch.cuda.stream(d2h):
+                y_h[b].copy_(y_d[b], non_blocking=True)
+                y_out[b].record(d2h)
+        stream.wait_event(y_out[(n - 1) & 1])
+        if n >= 2:
+            stream.wait_event(y_out[n & 1])
+        end.record(stream)
+        return start, end
 
-    with torch.cuda.stream(stream):
-        for _ in range(a.warmup):
-            e2e_step()
+    e2e_run(a.warmup)
     torch.cuda.synchronize()
     D.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(a.steps):
-            e2e_step()
-        e1.record(stream)
+    e0, e1 = e2e_run(a.steps)
     torch.cuda.synchronize()
     D.barrier()
     torch.cuda.synchronize()
     ms_e2e = D.max(e0.elapsed_time(e1))
+    if not torch.equal(y_h[(a.steps - 1) & 1], y.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident run")
     ck = clocks.stop(wall0, wall1, uuid) if clocks else None
 
     N = D.world
@@ -414,6 +450,7 @@ def ours_arm(a, D):
                        "groups": f"{cfg.n_groups}/{cfg.topk_groups}", "topk": cfg.topk,
                        "moe_inter": cfg.moe_inter, "shared_inter": cfg.shared_inter,
                        "score": cfg.score, "parallelism": f"replicas x{N}",
+                       "expert_kernel": a.expert_kernel,
                        "l2": "inputs larger than L2 (every step streams the active experts' "
                              f"weights, {n_active * 3 * cfg.moe_inter * cfg.dim * 2 / 1e9:.1f} GB)"},
             "e2e": {"value": e2e, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),

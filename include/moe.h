@@ -196,12 +196,23 @@ MOE_API moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void
 MOE_API moe_status moe_stage_timing_begin(int32_t max_calls);
 MOE_API int32_t moe_stage_timing_end(float* ms, int32_t n);
 
-/* Which kernel runs the expert GEMMs of a bf16 layer, process-wide:
- * AUTO (default) and TCGEN05 use the tensor-core grouped GEMM; SIMT uses the
- * CUDA-core grouped GEMM that fp32 layers always use. SIMT is a slow
- * independent cross-check of the tensor-core kernel, not a fallback: nothing
- * switches to it on its own. Returns MOE_ERR_INVALID_ARG for other values. */
-enum { MOE_EXPERT_KERNEL_AUTO = 0, MOE_EXPERT_KERNEL_SIMT = 1, MOE_EXPERT_KERNEL_TCGEN05 = 2 };
+/* Which kernels run the GEMMs of a bf16 layer, process-wide (for checks and
+ * measurement; nothing switches on its own):
+ *   AUTO (default)  tensor cores: router logits, and the grouped expert GEMM
+ *                   with one CTA per tile (128 rows) when experts average
+ *                   fewer than 128 rows, CTA pairs (256-row tiles) otherwise;
+ *   TCGEN05         tensor cores, expert GEMM always with one CTA per tile;
+ *   TCGEN05_PAIR    tensor cores, expert GEMM always on CTA pairs;
+ *   SIMT            the CUDA-core kernels that fp32 layers always use, for
+ *                   both the router logits and the expert GEMMs: a slow,
+ *                   independent cross-check of the tensor-core kernels.
+ * Returns MOE_ERR_INVALID_ARG for other values. */
+enum {
+  MOE_EXPERT_KERNEL_AUTO = 0,
+  MOE_EXPERT_KERNEL_SIMT = 1,
+  MOE_EXPERT_KERNEL_TCGEN05 = 2,
+  MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
+};
 MOE_API moe_status moe_select_expert_kernel(int32_t which);
 
 #ifdef __cplusplus

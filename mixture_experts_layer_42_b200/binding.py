@@ -29,6 +29,7 @@ MOE_ERR_TIMEOUT = -6
 MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX = 0, 1
 MOE_EXPERT_KERNEL_AUTO, MOE_EXPERT_KERNEL_SIMT, MOE_EXPERT_KERNEL_TCGEN05 = 0, 1, 2
+MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch",

@@ -172,9 +172,15 @@ struct GroupedArgs {
 // launcher calls it right after each kernel it launches.
 void stage_mark(cudaStream_t st);
 
+// Router: logits (tensor cores for bf16 unless `simt`, else CUDA cores) into
+// `part` with at most `splits` k splits, then selection into weights / idx.
 cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
                           const float* bias, float* weights, int32_t* idx, float* part,
-                          int splits, cudaStream_t st);
+                          int splits, bool simt, int num_sms, uint32_t* err, cudaStream_t st);
+int router_tc_splits(const moe_config& c, int64_t T, int max_splits, int num_sms);
+cudaError_t launch_router_logits_tc(const moe_config& c, int64_t T, const void* x,
+                                    const void* w_router, float* part, int splits, uint32_t* err,
+                                    cudaStream_t st, int* splits_used);
 // Built-in router scratch (moe_gate_noalloc): its size in floats, and its
 // device address on the current device.
 size_t gate_scratch_floats();
@@ -188,7 +194,7 @@ cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, c
                            const float* weights, const void* s, void* y, cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
-cudaError_t launch_grouped_tc(bool up, int64_t Tk, int64_t T_sh, int E, const void* a0,
+cudaError_t launch_grouped_tc(bool up, bool pair, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, uint32_t* err, int num_sms,

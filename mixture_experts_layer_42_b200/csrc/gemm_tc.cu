@@ -24,27 +24,13 @@
 // time share weight tiles and A rows in L2. Every pipeline wait is bounded
 // (1 s); on expiry the kernel raises the timeout bit of the error word, drains
 // what it has in flight, frees TMEM and returns.
-#include "common.cuh"
-
-#include <cuda.h>
-#include <cudaTypedefs.h>
+#include "tc_common.cuh"
 
 namespace moe {
 
-struct TcArgs {
-  CUtensorMap tmA[2];   // [0] routed A rows, [1] shared A rows; 2D {K, rows}
-  CUtensorMap tmB1[2];  // w1 (UP) / w2 (DOWN) as 3D {K, N, E}; shared: E = 1
-  CUtensorMap tmB3[2];  // w3 / ws3 (UP only)
-  void* out[2];
-  int n_out[2];         // output columns: UP I / I_s, DOWN D / D
-  int kdim[2];          // reduction depth: UP D / D, DOWN I / I_s
-  const int32_t* offsets;
-  int E;
-  int t_shared;         // rows of the shared group (0: none)
-  uint32_t* err;
-};
-
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128;
 constexpr int BK = 64;                     // one 128-byte swizzled row of bf16
@@ -55,130 +41,10 @@ constexpr int B_TILE = BN * BK * 2;        // 32 KB
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;   // 1 s
-constexpr uint64_t DRAIN_LIMIT_NS = 20000000ull;    // 20 ms
 constexpr int MAX_E = 1024;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * (MAX_E + 1) * 4;
 
-// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase of `bar` with the given parity. Gives up when another
-// role has raised the abort flag, or after WAIT_LIMIT_NS (then raises it).
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       uint32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
-      *abort_flag = 1;
-      set_error(err, ERRBIT_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// Bounded wait used only while draining after an abort.
-__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > DRAIN_LIMIT_NS) return;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, uint64_t* bar, int c0,
-                                            int c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, uint64_t* bar, int c0,
-                                            int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major tile written by TMA with the
-// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
+constexpr uint32_t IDESC = tc::idesc_bf16(BM, BN);
 
 struct Tile {
   int kind;   // 0 routed, 1 shared
@@ -358,7 +224,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
           const uint32_t b0 = a0 + A_TILE;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), (kb | kk) != 0 ? 1u : 0u);
+            tc_mma(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
           tc_commit(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
@@ -446,68 +312,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2D bf16 map over a row-major [rows, K] matrix, box 64 (K) x 128 rows.
-bool map_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
-  cuuint32_t box[2] = {BK, BM};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3D bf16 map over stacked weights [E, N, K], box 64 (K) x box_n x 1.
-bool map_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K,
-                 uint32_t box_n) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {K, N, E};
-  cuuint64_t strides[2] = {K * 2, N * K * 2};
-  cuuint32_t box[3] = {BK, box_n, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 // A: routed rows [Tk, K0] and shared rows [T, K1]; B1/B3 stacked [E, N0, K0]
-// and shared [N1, K1]; outputs [Tk, N0] and [T, N1].
-cudaError_t launch_grouped_tc(bool up, int64_t Tk, int64_t T_sh, int E, const void* a0,
+// and shared [N1, K1]; outputs [Tk, N0] and [T, N1]. `pair` selects the
+// CTA-pair kernel (256-row tiles, gemm_tc2.cu) instead of this one.
+cudaError_t launch_grouped_tc(bool up, bool pair, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, uint32_t* err, int num_sms,
                               cudaStream_t st) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
-  const uint32_t box_n = up ? BN / 2 : BN;
+  // B rows per TMA box: one CTA loads all 256 MMA rows (UP: 128 w1 + 128 w3);
+  // in a pair each CTA loads 128.
+  const uint32_t box_n = pair ? 128 : (up ? BN / 2 : BN);
   const bool has_sh = T_sh > 0;
-  if (!map_rows(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0)) return cudaErrorInvalidValue;
-  if (!map_weights(&g.tmB1[0], b1_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
+  if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, BM)) return cudaErrorInvalidValue;
+  if (!tc::map_3d(&g.tmB1[0], b1_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
-  if (up && !map_weights(&g.tmB3[0], b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
+  if (up && !tc::map_3d(&g.tmB3[0], b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (has_sh) {
-    if (!map_rows(&g.tmA[1], a1, (uint64_t)T_sh, (uint64_t)k1)) return cudaErrorInvalidValue;
-    if (!map_weights(&g.tmB1[1], b1_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
+    if (!tc::map_2d(&g.tmA[1], a1, (uint64_t)T_sh, (uint64_t)k1, BM)) return cudaErrorInvalidValue;
+    if (!tc::map_3d(&g.tmB1[1], b1_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
       return cudaErrorInvalidValue;
-    if (up && !map_weights(&g.tmB3[1], b3_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
+    if (up && !tc::map_3d(&g.tmB3[1], b3_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
       return cudaErrorInvalidValue;
   } else {
     g.tmA[1] = g.tmA[0];
@@ -526,16 +356,28 @@ cudaError_t launch_grouped_tc(bool up, int64_t Tk, int64_t T_sh, int E, const vo
   g.t_shared = has_sh ? (int)T_sh : 0;
   g.err = err;
 
+  // upper bound on the tiles (the exact count depends on the device offsets)
+  const int bm = pair ? 2 * BM : BM;
   const int bn_out = up ? BN / 2 : BN;
   const int64_t nt0 = (n0 + bn_out - 1) / bn_out;
-  const int64_t bound = nt0 * ((Tk + BM - 1) / BM + E) +
-                        (has_sh ? (int64_t)((n1 + bn_out - 1) / bn_out) * ((T_sh + BM - 1) / BM) : 0);
+  const int64_t bound = nt0 * ((Tk + bm - 1) / bm + E) +
+                        (has_sh ? (int64_t)((n1 + bn_out - 1) / bn_out) * ((T_sh + bm - 1) / bm) : 0);
+  cudaError_t e;
+  if (pair) {
+    const int pairs = (int)(bound < num_sms / 2 ? bound : num_sms / 2);
+    if (pairs <= 0) {
+      stage_mark(st);
+      return cudaSuccess;
+    }
+    e = launch_grouped_tc2(up, g, pairs, st);
+    stage_mark(st);
+    return e;
+  }
   const int grid = (int)(bound < num_sms ? bound : num_sms);
   if (grid <= 0) {
     stage_mark(st);
     return cudaSuccess;
   }
-  cudaError_t e;
   if (up) {
     e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);

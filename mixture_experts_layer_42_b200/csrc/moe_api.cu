@@ -96,11 +96,16 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
   if (tc) {
-    cudaError_t e = launch_grouped_tc(true, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
+    // CTA pairs (256-row tiles) pay off once experts average >= 128 rows;
+    // decode-sized batches stream weights with one CTA per SM.
+    bool pair = Tk >= (int64_t)128 * c.n_routed;
+    if (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05) pair = false;
+    if (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR) pair = true;
+    cudaError_t e = launch_grouped_tc(true, pair, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                                       c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
                                       err, num_sms_current(), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_grouped_tc(false, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
+    e = launch_grouped_tc(false, pair, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
                           c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, err,
                           num_sms_current(), st);
     return cuda_status(e);
@@ -182,7 +187,8 @@ moe_status moe_gate(const moe_config* cfg, int64_t T, const void* x, const void*
   if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
   return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx,
                                    at<float>(ws, L.router_part), L.router_splits,
-                                   (cudaStream_t)stream));
+                                   g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
+                                   at<uint32_t>(ws, L.header), (cudaStream_t)stream));
 }
 
 moe_status moe_dispatch(const moe_config* cfg, int64_t T, const int32_t* idx, const void* x,
@@ -275,7 +281,8 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   uint32_t* err = at<uint32_t>(ws, L.header);
   if (launch_router(c, T, x, w_router, bias, weights, idx, at<float>(ws, L.router_part),
-                    L.router_splits, s) != cudaSuccess)
+                    L.router_splits, g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
+                    err, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* pos = at<int32_t>(ws, L.pos);
@@ -342,7 +349,9 @@ moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, con
   int splits = router_splits(*cfg, T);
   const int64_t fit = (int64_t)gate_scratch_floats() / per_split;
   if (splits > fit) splits = (int)fit;
-  return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx, scratch, splits, s));
+  return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx, scratch, splits,
+                                   g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
+                                   nullptr, s));
 }
 
 moe_status moe_stage_timing_begin(int32_t max_calls) {
@@ -381,7 +390,7 @@ int32_t moe_stage_timing_end(float* ms, int32_t n) {
 
 moe_status moe_select_expert_kernel(int32_t which) {
   if (which != MOE_EXPERT_KERNEL_AUTO && which != MOE_EXPERT_KERNEL_SIMT &&
-      which != MOE_EXPERT_KERNEL_TCGEN05)
+      which != MOE_EXPERT_KERNEL_TCGEN05 && which != MOE_EXPERT_KERNEL_TCGEN05_PAIR)
     return MOE_ERR_INVALID_ARG;
   g_expert_kernel = which;
   return MOE_OK;

@@ -9,10 +9,11 @@
 //                         added into an fp64 accumulator, so the only rounding
 //                         that matters is the final cast of each split's sum
 //                         to fp32 (near-ties in routing depend on this).
-//   router_select_kernel  one warp per token: sums the splits (fp64, fixed
-//                         order), applies the score function, bias, group
-//                         limit and top-k with shuffle reductions, and writes
-//                         idx / weights.
+//   router_select_kernel  8 tokens per CTA: the CTA sums the splits (fp64,
+//                         fixed order) into shared memory, then one warp per
+//                         token applies the score function, bias, group limit
+//                         and top-k with shuffle reductions and writes idx /
+//                         weights.
 #include "common.cuh"
 
 #include <float.h>
@@ -172,21 +173,50 @@ struct SelectArgs {
 // Values per lane VPL = ceil(E / 32); expert e lives in lane e % 32, slot e / 32.
 template <int VPL>
 __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
+  extern __shared__ float z_s[];  // [8][E] logits of this CTA's tokens
   __shared__ float gsc_s[8][64];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-  if (t >= a.T) return;
   const int E = a.E;
+  const int64_t t0 = (int64_t)blockIdx.x * 8;
 
-  // 1. logits: fixed-order fp64 sum of the k splits, one fp32 rounding
+  // 1. logits: the CTA sums the k splits of its (up to) 8 tokens together --
+  //    each split's rows are one contiguous block of 8*E floats, and thread
+  //    i owns elements i + 256 q, q < VPL -- in fp64, in split order, with
+  //    one fp32 rounding, into shared memory. All VPL loads of a split are in
+  //    flight together.
+  {
+    const int64_t rows = a.T - t0 < 8 ? a.T - t0 : 8;
+    const int n = (int)(rows * E);
+    const int64_t stride = a.T * E;
+    const float* base = a.part + t0 * E;
+    double s[VPL];
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) s[q] = 0.0;
+#pragma unroll 2
+    for (int sp = 0; sp < a.splits; ++sp) {
+      float p[VPL];
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) {
+        const int i = threadIdx.x + 256 * q;
+        p[q] = i < n ? base[sp * stride + i] : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < VPL; ++q) s[q] += (double)p[q];
+    }
+#pragma unroll
+    for (int q = 0; q < VPL; ++q) {
+      const int i = threadIdx.x + 256 * q;
+      if (i < n) z_s[i] = (float)s[q];
+    }
+  }
+  __syncthreads();
+  const int64_t t = t0 + warp;
+  if (t >= a.T) return;
   float z[VPL];
 #pragma unroll
   for (int v = 0; v < VPL; ++v) {
-    int e = v * 32 + lane;
-    double sacc = 0.0;
-    if (e < E)
-      for (int sp = 0; sp < a.splits; ++sp) sacc += (double)a.part[((int64_t)sp * a.T + t) * E + e];
-    z[v] = (e < E) ? (float)sacc : -INFINITY;
+    const int e = v * 32 + lane;
+    z[v] = (e < E) ? z_s[warp * E + e] : -INFINITY;
   }
 
   // 2. scores (unbiased) and 3. selection scores
@@ -321,19 +351,30 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
 
 cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
                           const float* bias, float* weights, int32_t* idx, float* part,
-                          int splits, cudaStream_t st) {
+                          int splits, bool simt, int num_sms, uint32_t* err_word,
+                          cudaStream_t st) {
   const int E = c.n_routed, D = c.dim;
-  int kps = ceil_div(ceil_div(D, splits), RBK) * RBK;
-  splits = ceil_div(D, kps);
-  dim3 grid((unsigned)ceil_div<int64_t>(T, RBM), (unsigned)ceil_div(E, RBN), (unsigned)splits);
-  if (c.dtype == MOE_DT_BF16)
-    router_logits_kernel<__nv_bfloat16><<<grid, RTHREADS, 0, st>>>(
-        (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, T, E, D, kps, part);
-  else
-    router_logits_kernel<float><<<grid, RTHREADS, 0, st>>>((const float*)x, (const float*)w_router,
-                                                            T, E, D, kps, part);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
+  if (c.dtype == MOE_DT_BF16 && !simt) {
+    int used = 0;
+    err = launch_router_logits_tc(c, T, x, w_router, part, router_tc_splits(c, T, splits, num_sms),
+                                  err_word, st, &used);
+    if (err != cudaSuccess) return err;
+    splits = used;
+  } else {
+    const int kps = ceil_div(ceil_div(D, splits), RBK) * RBK;
+    splits = ceil_div(D, kps);
+    dim3 grid((unsigned)ceil_div<int64_t>(T, RBM), (unsigned)ceil_div(E, RBN), (unsigned)splits);
+    if (c.dtype == MOE_DT_BF16)
+      router_logits_kernel<__nv_bfloat16><<<grid, RTHREADS, 0, st>>>(
+          (const __nv_bfloat16*)x, (const __nv_bfloat16*)w_router, T, E, D, kps, part);
+    else
+      router_logits_kernel<float><<<grid, RTHREADS, 0, st>>>((const float*)x,
+                                                              (const float*)w_router, T, E, D, kps,
+                                                              part);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   stage_mark(st);
 
   SelectArgs a;
@@ -351,12 +392,13 @@ cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const v
   a.idx = idx;
   unsigned blocks = (unsigned)ceil_div<int64_t>(T, 8);
   int vpl = ceil_div(E, 32);
-  if (vpl <= 1) router_select_kernel<1><<<blocks, 256, 0, st>>>(a);
-  else if (vpl <= 2) router_select_kernel<2><<<blocks, 256, 0, st>>>(a);
-  else if (vpl <= 4) router_select_kernel<4><<<blocks, 256, 0, st>>>(a);
-  else if (vpl <= 8) router_select_kernel<8><<<blocks, 256, 0, st>>>(a);
-  else if (vpl <= 16) router_select_kernel<16><<<blocks, 256, 0, st>>>(a);
-  else router_select_kernel<32><<<blocks, 256, 0, st>>>(a);
+  const size_t zs = (size_t)8 * E * sizeof(float);
+  if (vpl <= 1) router_select_kernel<1><<<blocks, 256, zs, st>>>(a);
+  else if (vpl <= 2) router_select_kernel<2><<<blocks, 256, zs, st>>>(a);
+  else if (vpl <= 4) router_select_kernel<4><<<blocks, 256, zs, st>>>(a);
+  else if (vpl <= 8) router_select_kernel<8><<<blocks, 256, zs, st>>>(a);
+  else if (vpl <= 16) router_select_kernel<16><<<blocks, 256, zs, st>>>(a);
+  else router_select_kernel<32><<<blocks, 256, zs, st>>>(a);
   stage_mark(st);
   return cudaGetLastError();
 }

@@ -193,11 +193,30 @@ def _experts_case(cfg):
     return L, r, idx, w
 
 
-@pytest.mark.parametrize("kw", [{}, dict(T=640, dim=512, moe_inter=256), dict(moe_inter=200)])
-def test_tensor_core_experts_match_oracle(kw):
+class _kernel:
+    """Select the GEMM kernels for the duration of a block."""
+
+    def __init__(self, which):
+        self.which = which
+
+    def __enter__(self):
+        M.moe_select_expert_kernel(self.which)
+
+    def __exit__(self, *exc):
+        M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_AUTO)
+
+
+TC_KERNELS = [M.MOE_EXPERT_KERNEL_TCGEN05, M.MOE_EXPERT_KERNEL_TCGEN05_PAIR]
+
+
+@pytest.mark.parametrize("which", TC_KERNELS, ids=["one_cta", "cta_pair"])
+@pytest.mark.parametrize("kw", [{}, dict(T=640, dim=512, moe_inter=256), dict(moe_inter=200),
+                                dict(T=2000, n_routed=8, n_groups=2, topk_groups=1, topk=2)])
+def test_tensor_core_experts_match_oracle(kw, which):
     cfg = bf16_small(**kw)
     L, r, idx, w = _experts_case(cfg)
-    y, out = L.split(idx, w)
+    with _kernel(which):
+        y, out = L.split(idx, w)
     assert out["status"] == M.MOE_OK
     d = O.dispatch(r["idx"], cfg.n_routed)
     xp = host(out["x_perm"])
@@ -222,17 +241,31 @@ def test_tensor_core_vs_simt(kw):
     # fp32, so they agree far tighter than the layer tolerance
     cfg = bf16_small(**kw)
     L, r, idx, w = _experts_case(cfg)
-    y_tc, out_tc = L.split(idx, w)
-    M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_SIMT)
-    try:
+    with _kernel(M.MOE_EXPERT_KERNEL_SIMT):
         y_si, out_si = L.split(idx, w)
-    finally:
-        M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_AUTO)
-    a, b = to_np(out_tc["y_perm"]), to_np(out_si["y_perm"])
+    b = to_np(out_si["y_perm"])
     scale = np.abs(b).max()
-    assert np.abs(a - b).max() <= 2e-2 * scale
-    rel = np.abs(a - b) / (np.abs(b) + 1e-2 * scale)
-    assert np.median(rel) < 1e-2
+    for which in TC_KERNELS:
+        with _kernel(which):
+            y_tc, out_tc = L.split(idx, w)
+        a = to_np(out_tc["y_perm"])
+        assert np.abs(a - b).max() <= 2e-2 * scale
+        rel = np.abs(a - b) / (np.abs(b) + 1e-2 * scale)
+        assert np.median(rel) < 1e-2
+
+
+def test_pair_and_single_cta_kernels_agree_bitwise():
+    # the two tensor-core kernels add the same products in the same k order
+    # into fp32 accumulators, so their bf16 outputs are identical
+    cfg = bf16_small(T=1500, dim=512, moe_inter=256, n_routed=8, n_groups=2, topk_groups=1, topk=2)
+    L, r, idx, w = _experts_case(cfg)
+    outs = []
+    for which in TC_KERNELS:
+        with _kernel(which):
+            y, out = L.split(idx, w)
+        outs.append((y.cpu(), out["y_perm"].cpu(), out["s"].cpu()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
 
 
 def test_identity_experts_closed_form_gpu():
