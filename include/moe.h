@@ -199,8 +199,7 @@ MOE_API int32_t moe_stage_timing_end(float* ms, int32_t n);
 /* Which kernels run the GEMMs of a bf16 layer, process-wide (for checks and
  * measurement; nothing switches on its own):
  *   AUTO (default)  tensor cores: router logits, and the grouped expert GEMM
- *                   with one CTA per tile (128 rows) when experts average
- *                   fewer than 128 rows, CTA pairs (256-row tiles) otherwise;
+ *                   with one CTA per 128-row tile;
  *   TCGEN05         tensor cores, expert GEMM always with one CTA per tile;
  *   TCGEN05_PAIR    tensor cores, expert GEMM always on CTA pairs;
  *   SIMT            the CUDA-core kernels that fp32 layers always use, for

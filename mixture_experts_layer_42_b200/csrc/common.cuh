@@ -194,7 +194,9 @@ cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, c
                            const float* weights, const void* s, void* y, cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
-cudaError_t launch_grouped_tc(bool up, bool pair, int64_t Tk, int64_t T_sh, int E, const void* a0,
+// Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).
+enum { TC_ROWS = 0, TC_PAIR = 1 };
+cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, uint32_t* err, int num_sms,

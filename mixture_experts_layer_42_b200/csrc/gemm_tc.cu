@@ -16,8 +16,9 @@
 //               one tile overlaps the main loop of the next).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator rows (TMEM lane =
 //               tile row), silu(a)*b for UP, rounding to bf16, masked stores.
-// For UP the N=256 B tile stacks 128 rows of w1 over the same 128 rows of w3,
-// so accumulator columns j and 128+j hold a and b of the same feature.
+// For UP the N=256 B tile stacks 128 rows of w1 over the same 128 rows of w3
+// (one 4D TMA box over both tensors when their distance allows, else two
+// boxes), so accumulator columns j and 128+j hold a and b of the same feature.
 //
 // Tiles are enumerated from the device offsets (no host round trip): expert
 // by expert, n-tile outer and m-tile inner so that CTAs running at the same
@@ -185,7 +186,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
           uint8_t* sb = sa + A_TILE;
           mbar_expect_tx(&full[s], STAGE_BYTES);
           tma_load_2d(sa, &g.tmA[t.kind], &full[s], kb * BK, t.row0);
-          if (UP) {
+          if (UP && g.b13[t.kind]) {
+            tma_load_4d(sb, &g.tmB13[t.kind], &full[s], kb * BK, t.n0, t.e, 0);
+          } else if (UP) {
             tma_load_3d(sb, &g.tmB1[t.kind], &full[s], kb * BK, t.n0, t.e);
             tma_load_3d(sb + B_TILE / 2, &g.tmB3[t.kind], &full[s], kb * BK, t.n0, t.e);
           } else {
@@ -255,11 +258,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       __nv_bfloat16* out =
           reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]) + (int64_t)(t.row0 + row) * n_out + t.n0;
       if (UP) {
+        // accumulator columns of w1 (a) and w3 (b): w3 first when its tile
+        // came first in the paired load
+        const uint32_t ca = g.b13[t.kind] == 2 ? BN / 2 : 0, cb = BN / 2 - ca;
 #pragma unroll 1
         for (int j = 0; j < BN / 2; j += 16) {
           uint32_t ra[16], rb[16];
-          tmem_ld16(tb + j, ra);
-          tmem_ld16(tb + BN / 2 + j, rb);
+          tmem_ld16(tb + ca + j, ra);
+          tmem_ld16(tb + cb + j, rb);
           tmem_wait_ld();
           uint32_t pk[8];
 #pragma unroll
@@ -315,26 +321,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
 }  // namespace
 
 // A: routed rows [Tk, K0] and shared rows [T, K1]; B1/B3 stacked [E, N0, K0]
-// and shared [N1, K1]; outputs [Tk, N0] and [T, N1]. `pair` selects the
-// CTA-pair kernel (256-row tiles, gemm_tc2.cu) instead of this one.
-cudaError_t launch_grouped_tc(bool up, bool pair, int64_t Tk, int64_t T_sh, int E, const void* a0,
+// and shared [N1, K1]; outputs [Tk, N0] and [T, N1]. `kind` picks the
+// kernel: TC_ROWS this one (128-row tiles), TC_PAIR the CTA-pair kernel
+// (256-row tiles, gemm_tc2.cu).
+cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, uint32_t* err, int num_sms,
                               cudaStream_t st) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
-  // B rows per TMA box: one CTA loads all 256 MMA rows (UP: 128 w1 + 128 w3);
-  // in a pair each CTA loads 128.
+  const bool pair = kind == TC_PAIR;
+  // Weight rows per TMA box: one CTA loads all 256 MMA rows of B (UP: 128 w1
+  // + 128 w3); in a pair each CTA loads 128.
   const uint32_t box_n = pair ? 128 : (up ? BN / 2 : BN);
+  const uint32_t box_a = BM;
   const bool has_sh = T_sh > 0;
-  if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, BM)) return cudaErrorInvalidValue;
+  if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a)) return cudaErrorInvalidValue;
   if (!tc::map_3d(&g.tmB1[0], b1_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (up && !tc::map_3d(&g.tmB3[0], b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (has_sh) {
-    if (!tc::map_2d(&g.tmA[1], a1, (uint64_t)T_sh, (uint64_t)k1, BM)) return cudaErrorInvalidValue;
+    if (!tc::map_2d(&g.tmA[1], a1, (uint64_t)T_sh, (uint64_t)k1, box_a)) return cudaErrorInvalidValue;
     if (!tc::map_3d(&g.tmB1[1], b1_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
       return cudaErrorInvalidValue;
     if (up && !tc::map_3d(&g.tmB3[1], b3_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
@@ -345,6 +354,15 @@ cudaError_t launch_grouped_tc(bool up, bool pair, int64_t Tk, int64_t T_sh, int 
     g.tmB3[1] = g.tmB3[0];
   }
   if (!up) g.tmB3[0] = g.tmB1[0], g.tmB3[1] = g.tmB1[1];
+  // one-CTA UP: w1 and w3 tiles in one TMA box when the pair can be described
+  if (up && !pair) {
+    g.b13[0] = tc::map_pair_4d(&g.tmB13[0], b1_0, b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0,
+                               BN / 2);
+    if (has_sh)
+      g.b13[1] = tc::map_pair_4d(&g.tmB13[1], b1_1, b3_1, 1, (uint64_t)n1, (uint64_t)k1, BN / 2);
+    else
+      g.b13[1] = g.b13[0], g.tmB13[1] = g.tmB13[0];
+  }
   g.out[0] = out0;
   g.out[1] = has_sh ? out1 : out0;
   g.n_out[0] = n0;

@@ -96,16 +96,15 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
   if (tc) {
-    // CTA pairs (256-row tiles) pay off once experts average >= 128 rows;
-    // decode-sized batches stream weights with one CTA per SM.
-    bool pair = Tk >= (int64_t)128 * c.n_routed;
-    if (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05) pair = false;
-    if (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR) pair = true;
-    cudaError_t e = launch_grouped_tc(true, pair, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
+    // One CTA per 128-row tile unless CTA pairs are asked for: measured on
+    // the same GPU, the pairs' 256-row tiles pad enough extra rows at the
+    // DeepSeek-V3 prefill shape to lose to single CTAs under the power cap.
+    const int kind = g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR ? TC_PAIR : TC_ROWS;
+    cudaError_t e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                                       c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
                                       err, num_sms_current(), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_grouped_tc(false, pair, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
+    e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
                           c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, err,
                           num_sms_current(), st);
     return cuda_status(e);

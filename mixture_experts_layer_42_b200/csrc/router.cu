@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
     double s[VPL];
 #pragma unroll
     for (int q = 0; q < VPL; ++q) s[q] = 0.0;
-#pragma unroll 2
+#pragma unroll 4
     for (int sp = 0; sp < a.splits; ++sp) {
       float p[VPL];
 #pragma unroll

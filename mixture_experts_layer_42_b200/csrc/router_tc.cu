@@ -5,13 +5,17 @@
 // routing (near-ties at 1e-6) is the summation over D = 7168. So each 64-deep
 // k-block is accumulated by the tensor core into a fresh fp32 TMEM
 // accumulator (4 MMAs, 64 products per sum), and the epilogue warps add every
-// k-block's sums into fp64 registers. The tensor core therefore never sums
-// more than 64 products, and the result carries one fp32 rounding per split.
+// k-block's sums with Kahan's compensated summation in fp32 (sum plus a
+// running correction): its error stays within a few ulps of the sum however
+// many chunks are added, without fp64 work, at 4 additions per value.
+// The tensor core therefore never sums more than 64 products, and the result
+// carries one fp32 rounding per split.
 //
 // Tile: 128 tokens x 64 experts; grid (token tiles, expert tiles, k splits).
 // 192 threads: warp 0 TMA (x and W_r tiles, 128-byte swizzle, 4-stage ring),
-// warp 1 tcgen05.mma (M128 N64 K16) into two alternating 64-column TMEM
-// buffers, warps 2-5 tcgen05.ld + fp64 accumulation, then the split's
+// warp 1 tcgen05.mma (M128 N64 K16) into eight rotating 64-column TMEM
+// buffers (each k-block's sums wait there for the epilogue, so the MMA runs
+// up to eight k-blocks ahead), warps 2-5 tcgen05.ld + compensated accumulation, then the split's
 // partial logits are written as fp32 [split, T, E]. Waits are bounded as in
 // the expert GEMM kernel.
 #include "tc_common.cuh"
@@ -26,7 +30,8 @@ constexpr int RM = 128, RN = 64, RK = 64, RSTAGES = 4;
 constexpr int RA = RM * RK * 2;        // 16 KB x tile
 constexpr int RB = RN * RK * 2;        // 8 KB W_r tile
 constexpr int RSTAGE = RA + RB;
-constexpr uint32_t RTMEM = 128;        // two 64-column buffers
+constexpr int RNBUF = 8;               // TMEM chunk buffers between the MMA and the epilogue
+constexpr uint32_t RTMEM = RNBUF * RN; // 512 columns
 constexpr size_t RSMEM = 1024 + (size_t)RSTAGES * RSTAGE + 256;
 constexpr uint32_t RIDESC = idesc_bf16(RM, RN);
 
@@ -47,8 +52,8 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   uint64_t* full = reinterpret_cast<uint64_t*>(tiles + RSTAGES * RSTAGE);
   uint64_t* empty = full + RSTAGES;
   uint64_t* tfull = empty + RSTAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tempty = tfull + RNBUF;
+  uint64_t* drain = tempty + RNBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -62,7 +67,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < RSTAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+    for (int b = 0; b < RNBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -103,8 +108,8 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       int s = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nkb; ++i) {
-        const int b = i & 1;
-        const uint32_t use = (uint32_t)(i >> 1);
+        const int b = i % RNBUF;
+        const uint32_t use = (uint32_t)(i / RNBUF);
         if (!mbar_wait(&tempty[b], (use & 1) ^ 1, abort_flag, g.err)) break;
         tc_fence_after();
         if (!mbar_wait(&full[s], ph, abort_flag, g.err)) break;
@@ -125,13 +130,13 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   } else {
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    double acc[RN];
+    float hi[RN], lo[RN];
 #pragma unroll
-    for (int j = 0; j < RN; ++j) acc[j] = 0.0;
+    for (int j = 0; j < RN; ++j) hi[j] = lo[j] = 0.f;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
-      const int b = i & 1;
-      const uint32_t use = (uint32_t)(i >> 1);
+      const int b = i % RNBUF;
+      const uint32_t use = (uint32_t)(i / RNBUF);
       int w = 1;
       if (lane == 0) w = mbar_wait(&tfull[b], use & 1, abort_flag, g.err) ? 1 : 0;
       w = __shfl_sync(0xffffffffu, w, 0);
@@ -147,7 +152,12 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       tc_fence_before();
       mbar_arrive(&tempty[b]);
 #pragma unroll
-      for (int j = 0; j < RN; ++j) acc[j] += (double)__uint_as_float(r[j]);
+      for (int j = 0; j < RN; ++j) {  // Kahan: hi = running sum, lo = -(lost low part)
+        const float y = __fsub_rn(__uint_as_float(r[j]), lo[j]);
+        const float t = __fadd_rn(hi[j], y);
+        lo[j] = __fsub_rn(__fsub_rn(t, hi[j]), y);
+        hi[j] = t;
+      }
     }
     const int64_t t = (int64_t)m0 + row;
     if (ok && t < g.T) {
@@ -157,11 +167,12 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 #pragma unroll
         for (int j = 0; j < RN; j += 4)
           *reinterpret_cast<float4*>(out + j) =
-              make_float4((float)acc[j], (float)acc[j + 1], (float)acc[j + 2], (float)acc[j + 3]);
+              make_float4(__fsub_rn(hi[j], lo[j]), __fsub_rn(hi[j + 1], lo[j + 1]),
+                          __fsub_rn(hi[j + 2], lo[j + 2]), __fsub_rn(hi[j + 3], lo[j + 3]));
       } else {
 #pragma unroll
         for (int j = 0; j < RN; ++j)
-          if (j < nvalid) out[j] = (float)acc[j];
+          if (j < nvalid) out[j] = __fsub_rn(hi[j], lo[j]);
       }
     }
   }
@@ -177,13 +188,16 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 
 }  // namespace
 
-// Splits of the k range for T tokens: enough CTAs to cover the SMs, at most
-// `max_splits`, at least 4 k-blocks per split.
+// Splits of the k range for T tokens: about 32 CTAs for small batches --
+// the partial sums of every split are written out and summed again by the
+// select kernel, so more splits cost more than they hide -- at most
+// `max_splits`, at least 8 k-blocks per split.
 int router_tc_splits(const moe_config& c, int64_t T, int max_splits, int num_sms) {
+  (void)num_sms;
   const int64_t tiles = ceil_div<int64_t>(T, RM) * ceil_div<int64_t>(c.n_routed, RN);
   const int kbt = ceil_div(c.dim, RK);
-  int64_t s = ceil_div<int64_t>(num_sms, tiles);
-  if (s > kbt / 4) s = kbt / 4;
+  int64_t s = ceil_div<int64_t>(32, tiles);
+  if (s > kbt / 8) s = kbt / 8;
   if (s > max_splits) s = max_splits;
   if (s < 1) s = 1;
   return (int)s;

@@ -48,19 +48,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the thread sleep in hardware for up to ~1 us while the
+// phase is still pending, instead of spinning on the issue slots the other
+// warps of its SM sub-partition need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of `bar` with the given parity. Gives up when another
-// role has raised the abort flag, or after WAIT_LIMIT_NS (then raises it).
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       uint32_t* err) {
+// role has raised the abort flag, or after WAIT_LIMIT_NS (then raises it);
+// both are checked every 64 sleeping polls.
+static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, uint32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
-      *abort_flag = 1;
-      set_error(err, ERRBIT_TIMEOUT);
-      return false;
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((n & 63) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+        *abort_flag = 1;
+        set_error(err, ERRBIT_TIMEOUT);
+        return false;
+      }
     }
   }
 }
@@ -86,6 +104,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, ui
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
       "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, uint64_t* bar, int c0,
+                                            int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 
@@ -130,9 +157,75 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- CTA pairs
+// (cluster of two CTAs running tcgen05 cta_group::2 MMAs)
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `cta` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(cta));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on the
+// mbarrier at `bar` (a shared::cluster address, here the leader's).
+__device__ __forceinline__ void tma2_load_2d(void* dst, const CUtensorMap* tm, uint32_t bar, int c0,
+                                             int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma2_load_3d(void* dst, const CUtensorMap* tm, uint32_t bar, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the mbarrier at the same offset in both CTAs of the pair once
+// every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
+
 // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
 // K-major, the given M and N.
-constexpr uint32_t idesc_bf16(int M, int N) {
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -142,6 +235,12 @@ struct TcArgs {
   CUtensorMap tmA[2];   // [0] routed A rows, [1] shared A rows; 2D {K, rows}
   CUtensorMap tmB1[2];  // w1 (UP) / w2 (DOWN) as 3D {K, N, E}; shared: E = 1
   CUtensorMap tmB3[2];  // w3 / ws3 (UP only)
+  // UP only: w1 and w3 as one 4D map {K, N, E, 2} whose last stride is the
+  // distance between the two tensors, so one TMA box brings the w1 tile and
+  // the w3 tile; b13 = 0 when unavailable, 1 when w1 is the lower address
+  // (smem: w1 rows, then w3 rows), 2 when w3 is (smem: w3 rows, then w1).
+  CUtensorMap tmB13[2];
+  int b13[2];
   void* out[2];
   int n_out[2];         // output columns: UP I / I_s, DOWN D / D
   int kdim[2];          // reduction depth: UP D / D, DOWN I / I_s
@@ -154,6 +253,7 @@ struct TcArgs {
 // Launch the CTA-pair grouped GEMM (gemm_tc2.cu) on `pairs` clusters.
 cudaError_t launch_grouped_tc2(bool up, const TcArgs& g, int pairs, cudaStream_t st);
 
+
 // Host: TMA tensor-map encoder from the driver, without linking libcuda.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 
@@ -163,6 +263,13 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K, uint32_t
 
 // 3D bf16 map over stacked matrices [E, N, K], box 64 (K) x box_n x 1.
 bool map_3d(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K, uint32_t box_n);
+
+// 4D bf16 map over two same-shaped stacks [E, N, K] at p and q, box
+// 64 x box_n x 1 x 2 (the p tile then the q tile, or q then p when q is the
+// lower address). Returns 0 if the pair cannot be described (equal pointers,
+// or a distance TMA cannot stride), else 1 (p first) or 2 (q first).
+int map_pair_4d(CUtensorMap* m, const void* p, const void* q, uint64_t E, uint64_t N, uint64_t K,
+                uint32_t box_n);
 
 }  // namespace tc
 

@@ -295,3 +295,28 @@ def test_zero_w1_gives_shared_only_gpu():
     ws1, ws3, ws2 = L.w[3:]
     sref = O.swiglu(host(L.x), host(ws1), host(ws3), host(ws2), round_h="bf16", round_out="bf16")
     check_y(cfg, to_np(y), sref)
+
+
+@pytest.mark.parametrize("layout", ["w3_below_w1", "w1_is_w3", "one_buffer"])
+def test_w1_w3_memory_layouts(layout):
+    # the up-projection loads the w1 and w3 tiles with one TMA box over both
+    # tensors when their distance allows it, in either address order, and
+    # with two boxes otherwise: all three must give the oracle's layer
+    cfg = bf16_small(T=400)
+    L = Layer(cfg)
+    w1, w3, w2, ws1, ws3, ws2 = L.w
+    if layout == "w3_below_w1":
+        buf = torch.empty((2,) + tuple(w1.shape), dtype=w1.dtype, device="cuda")
+        buf[0].copy_(w3)
+        buf[1].copy_(w1)
+        sbuf = torch.empty((2,) + tuple(ws1.shape), dtype=ws1.dtype, device="cuda")
+        sbuf[0].copy_(ws3)
+        sbuf[1].copy_(ws1)
+        L.w = (buf[1], buf[0], w2, sbuf[1], sbuf[0], ws2)
+    elif layout == "w1_is_w3":
+        L.w = (w1, w1, w2, ws1, ws1, ws2)
+    else:  # w1 and w3 adjacent in one allocation, w1 first
+        buf = torch.stack([w1, w3])
+        L.w = (buf[0], buf[1], w2, ws1, ws3, ws2)
+    err, r, nt = forward_parity(L)
+    assert err < 2e-2
