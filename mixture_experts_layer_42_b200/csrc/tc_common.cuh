@@ -63,12 +63,11 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 
-// Wait for the phase of `bar` with the given parity. Gives up when another
-// role has raised the abort flag, or after WAIT_LIMIT_NS (then raises it);
-// both are checked every 64 sleeping polls.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag, uint32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: poll with sleeping try_waits, giving up when
+// another role has raised the abort flag or after WAIT_LIMIT_NS (then raises
+// it); both are checked every 64 polls.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity,
+                                                   volatile int* abort_flag, uint32_t* err) {
   const uint64_t t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
@@ -81,6 +80,15 @@ static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
       }
     }
   }
+}
+
+// Wait for the phase of `bar` with the given parity (bounded, see
+// mbar_wait_slow). The first try is inline: on the pipeline's critical path
+// the phase has usually completed already.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, err);
 }
 
 // Bounded wait used only while draining after an abort.
