@@ -82,16 +82,24 @@ def workload(a):
 # ---------------------------------------------------------------- distributed
 
 class Dist:
-    def __init__(self):
+    """One process per GPU (torchrun env). The layer does not shard: ranks run
+    independent replicas and only meet for the timing barrier and the max of
+    the per-rank device times (NCCL on GPUs, gloo when there are none)."""
+
+    def __init__(self, backend=None):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = False
         if self.world > 1:
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+            self.dev = torch.device("cuda", self.local) if backend == "nccl" else torch.device("cpu")
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = self.dev
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = True
 
     def barrier(self):
@@ -103,7 +111,7 @@ class Dist:
         if not self.pg:
             return v
         import torch.distributed as dist
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device=self.dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -469,6 +477,9 @@ def ours_arm(a, D):
 def main():
     a = parse()
     D = Dist()
+    if D.world != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but {D.world} process(es) were launched "
+                         "(use torchrun --nproc-per-node N for N > 1)")
     try:
         if a.impl == "reference":
             reference_arm(a, D)
