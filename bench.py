@@ -314,10 +314,10 @@ def ours_arm(a, D):
     ws = M.alloc_workspace(cfg, T, dev)
     torch.cuda.synchronize()
     stream = torch.cuda.Stream(device=dev)
-    launches = M.moe_forward_launch_count(cfg, T)
     M.moe_select_expert_kernel({"auto": M.MOE_EXPERT_KERNEL_AUTO, "simt": M.MOE_EXPERT_KERNEL_SIMT,
                                 "one_cta": M.MOE_EXPERT_KERNEL_TCGEN05,
                                 "pair": M.MOE_EXPERT_KERNEL_TCGEN05_PAIR}[a.expert_kernel])
+    launches = M.moe_forward_launch_count(cfg, T)
 
     def step(xin=x, idx_out=None):
         M.moe_forward(cfg, xin, w_r, bias, *w, y, ws, idx_out=idx_out, stream=stream)

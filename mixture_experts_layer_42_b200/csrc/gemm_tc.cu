@@ -180,12 +180,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       for (int i = blockIdx.x; ok && i < S.total; i += gridDim.x) {
         const Tile t = decode(S, i);
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
+        // an expert's last tile reads zeros past its rows, not the next
+        // expert's (the padding rows then cost the tensor cores less power)
+        const CUtensorMap* ta = &g.tmA[t.kind];
+        if (t.kind == 0 && t.rows < BM && g.row_maps != nullptr) {
+          ta = g.row_maps + t.e;
+          tmap_acquire(ta);
+        }
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err)) { ok = false; break; }
           uint8_t* sa = tiles + s * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
           mbar_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_2d(sa, &g.tmA[t.kind], &full[s], kb * BK, t.row0);
+          tma_load_2d(sa, ta, &full[s], kb * BK, t.row0);
           if (UP && g.b13[t.kind]) {
             tma_load_4d(sb, &g.tmB13[t.kind], &full[s], kb * BK, t.n0, t.e, 0);
           } else if (UP) {
@@ -318,6 +325,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   }
 }
 
+// Per-expert copies of the routed A map with the row extent cut at the
+// expert's end: one warp per expert edits a copy in shared memory and
+// publishes it to global memory with a release fence for the tensor-map proxy.
+__global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ CUtensorMap base,
+                                                             const int32_t* __restrict__ offsets,
+                                                             int E, CUtensorMap* maps) {
+  __shared__ __align__(128) CUtensorMap sm[8];
+  const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int e = blockIdx.x * 8 + w;
+  if (e >= E) return;  // whole warps
+  reinterpret_cast<uint32_t*>(&sm[w])[lane] = reinterpret_cast<const uint32_t*>(&base)[lane];
+  __syncwarp();
+  if (lane == 0) {
+    const int end = offsets[e + 1];
+    asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], 1, %1;" ::"r"(
+                     smem_u32(&sm[w])),
+                 "r"(end > 0 ? end : 1)
+                 : "memory");
+  }
+  __syncwarp();
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], "
+      "[%1], 128;" ::"l"(maps + e),
+      "r"(smem_u32(&sm[w]))
+      : "memory");
+}
+
 }  // namespace
 
 // A: routed rows [Tk, K0] and shared rows [T, K1]; B1/B3 stacked [E, N0, K0]
@@ -327,39 +361,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
-                              void* out1, const int32_t* offsets, uint32_t* err, int num_sms,
-                              cudaStream_t st) {
+                              void* out1, const int32_t* offsets, void* row_maps, uint32_t* err,
+                              int num_sms, cudaStream_t st) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
   const bool pair = kind == TC_PAIR;
   // Weight rows per TMA box: one CTA loads all 256 MMA rows of B (UP: 128 w1
-  // + 128 w3); in a pair each CTA loads 128.
-  const uint32_t box_n = pair ? 128 : (up ? BN / 2 : BN);
+  // + 128 w3); in a pair each CTA loads 128 (UP: 64 w1 + 64 w3).
+  const uint32_t box_n = up ? (pair ? BN / 4 : BN / 2) : (pair ? BN / 2 : BN);
   const uint32_t box_a = BM;
   const bool has_sh = T_sh > 0;
   if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a)) return cudaErrorInvalidValue;
+  if (pair && !tc::map_2d(&g.tmA64[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a / 2))
+    return cudaErrorInvalidValue;
   if (!tc::map_3d(&g.tmB1[0], b1_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (up && !tc::map_3d(&g.tmB3[0], b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (has_sh) {
     if (!tc::map_2d(&g.tmA[1], a1, (uint64_t)T_sh, (uint64_t)k1, box_a)) return cudaErrorInvalidValue;
+    if (pair && !tc::map_2d(&g.tmA64[1], a1, (uint64_t)T_sh, (uint64_t)k1, box_a / 2))
+      return cudaErrorInvalidValue;
     if (!tc::map_3d(&g.tmB1[1], b1_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
       return cudaErrorInvalidValue;
     if (up && !tc::map_3d(&g.tmB3[1], b3_1, 1, (uint64_t)n1, (uint64_t)k1, box_n))
       return cudaErrorInvalidValue;
   } else {
     g.tmA[1] = g.tmA[0];
+    g.tmA64[1] = g.tmA64[0];
     g.tmB1[1] = g.tmB1[0];
     g.tmB3[1] = g.tmB3[0];
   }
   if (!up) g.tmB3[0] = g.tmB1[0], g.tmB3[1] = g.tmB1[1];
-  // one-CTA UP: w1 and w3 tiles in one TMA box when the pair can be described
-  if (up && !pair) {
+  // UP: w1 and w3 tiles in one TMA box when the two tensors can be described
+  // by one map
+  if (up) {
     g.b13[0] = tc::map_pair_4d(&g.tmB13[0], b1_0, b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0,
-                               BN / 2);
+                               box_n);
     if (has_sh)
-      g.b13[1] = tc::map_pair_4d(&g.tmB13[1], b1_1, b3_1, 1, (uint64_t)n1, (uint64_t)k1, BN / 2);
+      g.b13[1] = tc::map_pair_4d(&g.tmB13[1], b1_1, b3_1, 1, (uint64_t)n1, (uint64_t)k1, box_n);
     else
       g.b13[1] = g.b13[0], g.tmB13[1] = g.tmB13[0];
   }
@@ -395,6 +435,13 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
   if (grid <= 0) {
     stage_mark(st);
     return cudaSuccess;
+  }
+  if (row_maps != nullptr && E > 0) {
+    g.row_maps = static_cast<const CUtensorMap*>(row_maps);
+    build_row_maps_kernel<<<(E + 7) / 8, 256, 0, st>>>(g.tmA[0], offsets, E,
+                                                       static_cast<CUtensorMap*>(row_maps));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
   if (up) {
     e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -2,17 +2,26 @@
 // batches with many rows per expert (prefill).
 //
 // Same layer math and tile order as the one-CTA kernel (gemm_tc.cu), with a
-// 256-row tile computed by a cluster of two CTAs on neighbouring SMs:
-//   * each CTA's TMA warp loads ITS 128 rows of A and ITS 128-row half of the
-//     N=256 B tile (UP: rank 0 loads the w1 rows, rank 1 the same w3 rows;
-//     DOWN: rank r loads output columns [n0 + 128 r, n0 + 128 r + 128)) into
-//     its own 6-stage ring. Both CTAs' copies signal the leader's (rank 0)
-//     "full" barrier; no load is multicast.
-//   * the leader's MMA thread issues tcgen05.mma.cta_group::2 M=256 N=256
-//     K=16, reading the two halves of A and B from the two CTAs' shared
-//     memory at the same offsets; each CTA's TMEM receives its 128 rows x 256
-//     fp32 columns. Commits are multicast to both CTAs' barriers.
-//   * each CTA's epilogue warps drain their own TMEM rows (silu(a)*b for UP)
+// tile of up to 256 rows computed by a cluster of two CTAs on neighbouring
+// SMs:
+//   * each CTA's TMA warp loads its share of A and its 128-row half of the
+//     N=256 B tile into its own 6-stage ring (UP: rank r loads rows
+//     [n0 + 64 r, n0 + 64 r + 64) of w1 and the same rows of w3, so every
+//     half holds a and b of the same 64 features; DOWN: rank r loads output
+//     columns [n0 + 128 r, n0 + 128 r + 128)). Both CTAs' copies signal the
+//     leader's (rank 0) "full" barrier; no load is multicast.
+//   * the leader's MMA thread issues tcgen05.mma.cta_group::2 K=16, N=256:
+//       - M=256 while more than 128 rows of the tile are valid: each CTA
+//         holds 128 A rows and its TMEM lane l = tile row 128 r + l, with
+//         columns 0-255 = the N columns;
+//       - M=128 for an expert's last chunk of at most 128 rows (its padding is
+//         then that of 128-row tiles): each CTA holds 64 A rows; TMEM lanes
+//         0-63 hold those rows against N columns 0-127 (the leader's B half),
+//         lanes 64-127 the same rows against N columns 128-255, both in TMEM
+//         columns 0-127.
+//     M=128 on a pair runs at nearly the M=256 rate per FLOP (unlike M=64 on
+//     one CTA, which runs at half rate). Commits are multicast to both CTAs.
+//   * each CTA's epilogue warps drain their own TMEM lanes (silu(a)*b for UP)
 //     and arrive on the leader's accumulator-free barrier.
 // Per CTA a stage is 32 KB instead of 48 KB for the same MMA work, so six
 // stages fit, and each B byte is read once per 256 rows instead of 128.
@@ -37,7 +46,9 @@ constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * (MAX_E + 1) * 4;
-constexpr uint32_t IDESC = idesc_bf16(PBM, BN);
+constexpr uint32_t IDESC = idesc_bf16(PBM, BN);       // full chunk: 256 rows
+constexpr uint32_t IDESC_TAIL = idesc_bf16(HBM, BN);  // last chunk of <= 128 rows
+constexpr int A_TAIL = HBM / 2 * BK * 2;              // 8 KB: 64 A rows per CTA
 
 struct Tile {
   int kind, e, row0, rows, n0;
@@ -172,16 +183,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       for (int i = pair; ok && i < S.total; i += npairs) {
         const Tile t = decode(S, i);
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
-        const int arow = t.row0 + (int)rank * HBM;
-        const int brow = UP ? t.n0 : t.n0 + (int)rank * HBN;
-        const CUtensorMap* tb = (UP && rank == 1) ? &g.tmB3[t.kind] : &g.tmB1[t.kind];
+        const bool tail = t.rows <= HBM;
+        const CUtensorMap* ta = tail ? &g.tmA64[t.kind] : &g.tmA[t.kind];
+        const int arow = t.row0 + (int)rank * (tail ? HBM / 2 : HBM);
+        const uint32_t tx = 2u * (uint32_t)((tail ? A_TAIL : A_HALF) + B_HALF);
+        // UP: w1 and w3 rows [n0 + 64 r, +64); DOWN: output columns [n0 + 128 r, +128)
+        const int brow = UP ? t.n0 + (int)rank * (HBN / 2) : t.n0 + (int)rank * HBN;
+        const int b13 = UP ? g.b13[t.kind] : 0;
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err)) { ok = false; break; }
           uint8_t* sa = tiles + s * STAGE_BYTES;
           const uint32_t fb = mapa(smem_u32(&full[s]), 0);
-          if (leader) mbar_expect_tx(&full[s], 2 * STAGE_BYTES);
-          tma2_load_2d(sa, &g.tmA[t.kind], fb, kb * BK, arow);
-          tma2_load_3d(sa + A_HALF, tb, fb, kb * BK, brow, t.e);
+          if (leader) mbar_expect_tx(&full[s], tx);
+          tma2_load_2d(sa, ta, fb, kb * BK, arow);
+          if (!UP) {
+            tma2_load_3d(sa + A_HALF, &g.tmB1[t.kind], fb, kb * BK, brow, t.e);
+          } else if (b13 != 0) {
+            tma2_load_4d(sa + A_HALF, &g.tmB13[t.kind], fb, kb * BK, brow, t.e, 0);
+          } else {
+            tma2_load_3d(sa + A_HALF, &g.tmB1[t.kind], fb, kb * BK, brow, t.e);
+            tma2_load_3d(sa + A_HALF + B_HALF / 2, &g.tmB3[t.kind], fb, kb * BK, brow, t.e);
+          }
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
@@ -201,6 +223,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       for (int i = pair; ok && i < S.total; i += npairs, ++lt) {
         const Tile t = decode(S, i);
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
+        const uint32_t idesc = t.rows <= HBM ? IDESC_TAIL : IDESC;
         const int acc = lt & 1;
         const uint32_t use = (uint32_t)(lt >> 1);
         if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, g.err)) break;
@@ -213,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b0 = a0 + A_HALF;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_pair(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
+            mma_pair(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
           commit_pair(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
@@ -240,17 +263,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
-      const int my_row = (int)rank * HBM + row;
+      const bool tail = t.rows <= HBM;
+      // tile row held by this lane, and the first N column of its TMEM column 0
+      const int my_row = tail ? (int)rank * (HBM / 2) + (row & (HBM / 2 - 1)) : (int)rank * HBM + row;
+      const int ncol0 = tail ? (row / (HBM / 2)) * (BN / 2) : 0;
+      const int ncols = tail ? BN / 2 : BN;  // TMEM columns holding this lane's results (DOWN)
       const bool valid = my_row < t.rows;
       const int n_out = g.n_out[t.kind];
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]) +
                            (int64_t)(t.row0 + my_row) * n_out + t.n0;
       if (UP) {
+        // every 128 N columns hold 64 features: 64 w1 rows, then the same 64
+        // w3 rows (b13 = 2: w3 first). Full chunk: 128 features in TMEM
+        // columns 0-255; tail: this lane's 64 features in columns 0-127.
+        const int ca = g.b13[t.kind] == 2 ? BN / 4 : 0;
+        const int cb = BN / 4 - ca;
+        const int nfeat = tail ? BN / 4 : BN / 2;
+        const int f0 = ncol0 / 2;
 #pragma unroll 1
-        for (int j = 0; j < BN / 2; j += 16) {
+        for (int u = 0; u < nfeat; u += 16) {
+          const int f = f0 + u;                       // feature offset from n0
+          const int col = (u / (BN / 4)) * (BN / 2) + (u % (BN / 4));
           uint32_t ra[16], rb[16];
-          tmem_ld16(tb + j, ra);
-          tmem_ld16(tb + BN / 2 + j, rb);
+          tmem_ld16(tb + col + ca, ra);
+          tmem_ld16(tb + col + cb, rb);
           tmem_wait_ld();
           uint32_t pk[8];
 #pragma unroll
@@ -262,17 +298,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             pk[q] = *reinterpret_cast<uint32_t*>(&v);
           }
           if (valid) {
-            if (t.n0 + j + 8 <= n_out)
-              *reinterpret_cast<uint4*>(out + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            if (t.n0 + j + 16 <= n_out)
-              *reinterpret_cast<uint4*>(out + j + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (t.n0 + f + 8 <= n_out)
+              *reinterpret_cast<uint4*>(out + f) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (t.n0 + f + 16 <= n_out)
+              *reinterpret_cast<uint4*>(out + f + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
       } else {
 #pragma unroll 1
-        for (int j = 0; j < BN; j += 16) {
+        for (int c = 0; c < ncols; c += 16) {
           uint32_t ra[16];
-          tmem_ld16(tb + j, ra);
+          tmem_ld16(tb + c, ra);
           tmem_wait_ld();
           uint32_t pk[8];
 #pragma unroll
@@ -281,11 +317,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 __floats2bfloat162_rn(__uint_as_float(ra[2 * q]), __uint_as_float(ra[2 * q + 1]));
             pk[q] = *reinterpret_cast<uint32_t*>(&v);
           }
+          const int n = ncol0 + c;
           if (valid) {
-            if (t.n0 + j + 8 <= n_out)
-              *reinterpret_cast<uint4*>(out + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            if (t.n0 + j + 16 <= n_out)
-              *reinterpret_cast<uint4*>(out + j + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (t.n0 + n + 8 <= n_out)
+              *reinterpret_cast<uint4*>(out + n) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (t.n0 + n + 16 <= n_out)
+              *reinterpret_cast<uint4*>(out + n + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
       }

@@ -91,7 +91,7 @@ moe_status bind_device(cudaStream_t s, const void* ptr) {
 moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* offsets,
                        const void* w1, const void* w3, const void* w2, const void* x,
                        const void* ws1, const void* ws3, const void* ws2, void* y_perm, void* s,
-                       void* h, void* hs, uint32_t* err, cudaStream_t st) {
+                       void* h, void* hs, void* row_maps, uint32_t* err, cudaStream_t st) {
   const int64_t Tk = T * c.topk;
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
@@ -102,10 +102,11 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
     const int kind = g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR ? TC_PAIR : TC_ROWS;
     cudaError_t e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                                       c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
-                                      err, num_sms_current(), st);
+                                      row_maps, err, num_sms_current(), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
-                          c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, err,
+                          c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets,
+                          static_cast<uint8_t*>(row_maps) + (size_t)c.n_routed * 128, err,
                           num_sms_current(), st);
     return cuda_status(e);
   }
@@ -223,8 +224,8 @@ moe_status moe_experts_grouped(const moe_config* cfg, int64_t T, const void* x_p
   if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
   if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
   return run_experts(*cfg, T, x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, y_perm, s,
-                     at<void>(ws, L.h), at<void>(ws, L.hs), at<uint32_t>(ws, L.header),
-                     (cudaStream_t)stream);
+                     at<void>(ws, L.h), at<void>(ws, L.hs), at<void>(ws, L.row_maps),
+                     at<uint32_t>(ws, L.header), (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_perm, const int32_t* pos,
@@ -292,7 +293,8 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
   st = run_experts(c, T, at<void>(ws, L.x_perm), offsets, w1, w3, w2, x, ws1, ws3, ws2,
-                   at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs), err, s);
+                   at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
+                   at<void>(ws, L.row_maps), err, s);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
 }
@@ -328,8 +330,11 @@ const char* moe_status_string(moe_status st) {
 int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
   if (check_config(cfg, T) != MOE_OK) return -1;
   // router: logits + select; dispatch: rank + scan + scatter; experts: up +
-  // down; combine
-  return 2 + 3 + 2 + 1;
+  // down, each after a kernel that writes its per-expert A maps when the
+  // one-CTA tensor-core kernel runs; combine
+  const bool row_maps = cfg->dtype == MOE_DT_BF16 && (g_expert_kernel == MOE_EXPERT_KERNEL_AUTO ||
+                                                      g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05);
+  return 2 + 3 + 2 + (row_maps ? 2 : 0) + 1;
 }
 
 moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, const void* w_router,

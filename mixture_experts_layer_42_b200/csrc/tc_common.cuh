@@ -124,6 +124,12 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, ui
       : "memory");
 }
 
+// Make a tensor map written to global memory through the generic proxy
+// (tensormap.cp_fenceproxy ... release) visible to this thread's TMA loads.
+__device__ __forceinline__ void tmap_acquire(const void* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -205,6 +211,15 @@ __device__ __forceinline__ void tma2_load_3d(void* dst, const CUtensorMap* tm, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma2_load_4d(void* dst, const CUtensorMap* tm, uint32_t bar, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -241,18 +256,24 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 // experts (A rows expert-contiguous, B stacked per expert), [1] the shared MLP.
 struct TcArgs {
   CUtensorMap tmA[2];   // [0] routed A rows, [1] shared A rows; 2D {K, rows}
+  CUtensorMap tmA64[2]; // the same with 64-row boxes (CTA-pair tail chunks)
   CUtensorMap tmB1[2];  // w1 (UP) / w2 (DOWN) as 3D {K, N, E}; shared: E = 1
   CUtensorMap tmB3[2];  // w3 / ws3 (UP only)
   // UP only: w1 and w3 as one 4D map {K, N, E, 2} whose last stride is the
   // distance between the two tensors, so one TMA box brings the w1 tile and
   // the w3 tile; b13 = 0 when unavailable, 1 when w1 is the lower address
   // (smem: w1 rows, then w3 rows), 2 when w3 is (smem: w3 rows, then w1).
+  // Boxes hold 128 rows of each for one CTA, 64 for a CTA pair.
   CUtensorMap tmB13[2];
   int b13[2];
   void* out[2];
   int n_out[2];         // output columns: UP I / I_s, DOWN D / D
   int kdim[2];          // reduction depth: UP D / D, DOWN I / I_s
   const int32_t* offsets;
+  // One-CTA kernel: [E] copies of tmA[0] whose row extent ends at the
+  // expert's last row (offsets[e + 1]), so that a tile reaching past it reads
+  // zeros there; null when not built.
+  const CUtensorMap* row_maps;
   int E;
   int t_shared;         // rows of the shared group (0: none)
   uint32_t* err;

@@ -116,5 +116,13 @@ def test_workspace_size_grows_with_tokens(M):
 
 
 def test_launch_count(M):
-    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 8
+    # bf16 on the one-CTA tensor-core kernel: each expert GEMM follows a
+    # kernel that writes its per-expert A maps
+    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 10
+    assert M.moe_forward_launch_count(inputs.CONFIGS["tiny_fp32"], 64) == 8
+    M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_TCGEN05_PAIR)
+    try:
+        assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 8
+    finally:
+        M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_AUTO)
     assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 0) == -1
