@@ -467,7 +467,11 @@ def ours_arm(a, D):
             "roofline": roof,
             "layer_roofline": {"flops": flops, "bytes": byts, "bound": bound,
                                "t_roofline_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_step,
-                               "peak_source": pk_kind},
+                               "peak_source": f"{pk_kind} (burst)",
+                               # the same against the seconds-long (power-capped) GEMM peak
+                               "frac_sustained": layer_roofline(
+                                   cfg, n_active, dict(pk, bf16_tflops=pk["bf16_tflops_sustained"]))[2]
+                               * 1e3 / ms_step},
             "kernels_ms": per_kernel_ms, "dominant_kernel": dom, "active_experts": n_active,
             "cpu_baseline": cpu, "clocks": ck,
         }
