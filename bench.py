@@ -327,7 +327,13 @@ def ours_arm(a, D):
     torch.cuda.synchronize()
     if M.moe_check_error(ws, stream) != M.MOE_OK:
         raise RuntimeError("device error word set after the first forward")
-    n_active = int((torch.bincount(idx.flatten().long(), minlength=cfg.n_routed) > 0).sum().item())
+    counts = torch.bincount(idx.flatten().long(), minlength=cfg.n_routed).cpu()
+    n_active = int((counts > 0).sum().item())
+    routing = {"active_experts": n_active, "max_count": int(counts.max()), "min_count": int(counts.min()),
+               "mean_count": T * cfg.topk / cfg.n_routed,
+               "rows_useful_in_128_row_tiles": float(counts.sum() / (128 * ((counts + 127) // 128).sum()))}
+    if cfg.name == "v3_zipf":
+        routing.update(zipf_s=inputs.ZIPF_S, zipf_beta=inputs.ZIPF_BETA)
 
     uuid = None
     try:
@@ -473,6 +479,7 @@ def ours_arm(a, D):
                                    cfg, n_active, dict(pk, bf16_tflops=pk["bf16_tflops_sustained"]))[2]
                                * 1e3 / ms_step},
             "kernels_ms": per_kernel_ms, "dominant_kernel": dom, "active_experts": n_active,
+            "routing": routing,
             "cpu_baseline": cpu, "clocks": ck,
         }
         print(json.dumps(line), flush=True)

@@ -320,3 +320,11 @@ def test_w1_w3_memory_layouts(layout):
         L.w = (buf[0], buf[1], w2, ws1, ws3, ws2)
     err, r, nt = forward_parity(L)
     assert err < 2e-2
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "softmax_nogroup"])
+def test_routing_profile_driver_runs(name, capsys):
+    # the profiling driver of the non-expert kernels (no expert weights)
+    from mixture_experts_layer_42_b200 import profile_routing
+    profile_routing.main(["--config", name, "--iters", "2"])
+    assert "done" in capsys.readouterr().out
