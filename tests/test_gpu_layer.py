@@ -40,6 +40,8 @@ def test_tiny_fp32_forward_all_tokens():
     dict(n_routed=64, n_groups=8, topk_groups=3, topk=6, moe_inter=136),
     dict(n_shared=0),
     dict(T=513, dim=1024, moe_inter=512, n_routed=32, n_groups=4, topk_groups=2, topk=8),
+    # the most experts and picks the library accepts: 1024 experts, top-32
+    dict(T=200, dim=256, moe_inter=128, n_routed=1024, n_groups=32, topk_groups=8, topk=32),
 ])
 def test_bf16_forward_all_tokens(kw):
     err, r, nt = forward_parity(Layer(bf16_small(**kw)))
@@ -76,6 +78,31 @@ def test_gate_all_tokens(name):
     r = L.oracle_route()
     differs = check_routing(cfg, idx, wts, r)
     assert differs.sum() <= max(2, L.T // 1000)
+
+
+@pytest.mark.parametrize("kw", [
+    # the largest routing shapes the library accepts, and unusual group widths
+    dict(n_routed=1024, n_groups=32, topk_groups=8, topk=32),            # 32 experts per group
+    dict(n_routed=1024, n_groups=64, topk_groups=16, topk=8),            # 16 per group
+    dict(n_routed=1024, n_groups=1, topk_groups=1, topk=32, score="softmax", bias="none"),
+    dict(n_routed=8, n_groups=4, topk_groups=2, topk=4),                 # 2 per group (top-2 = both)
+    dict(n_routed=96, n_groups=3, topk_groups=2, topk=6),                # E not a power of two
+    dict(n_routed=48, n_groups=3, topk_groups=1, topk=16),               # k = the whole kept group
+    dict(n_routed=512, n_groups=8, topk_groups=4, topk=1),               # k = 1
+    dict(n_routed=64, n_groups=2, topk_groups=2, topk=8),                # every group kept
+])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_gate_routing_limits(kw, dtype):
+    cfg = bf16_small(T=333, dim=512, dtype=dtype, **kw)
+    L = Layer(cfg, weights=(None,) * 6)
+    wts = torch.empty(L.T, cfg.topk, dtype=torch.float32, device="cuda")
+    idx = torch.empty(L.T, cfg.topk, dtype=torch.int32, device="cuda")
+    ws = M.alloc_workspace(cfg, L.T)
+    M.moe_gate(cfg, L.x, L.w_r, L.bias, wts, idx, ws)
+    torch.cuda.synchronize()
+    r = L.oracle_route()
+    differs = check_routing(cfg, idx, wts, r)
+    assert differs.sum() <= 2
 
 
 def test_gate_zero_router_closed_form():
@@ -211,7 +238,9 @@ TC_KERNELS = [M.MOE_EXPERT_KERNEL_TCGEN05, M.MOE_EXPERT_KERNEL_TCGEN05_PAIR]
 
 @pytest.mark.parametrize("which", TC_KERNELS, ids=["one_cta", "cta_pair"])
 @pytest.mark.parametrize("kw", [{}, dict(T=640, dim=512, moe_inter=256), dict(moe_inter=200),
-                                dict(T=2000, n_routed=8, n_groups=2, topk_groups=1, topk=2)])
+                                dict(T=2000, n_routed=8, n_groups=2, topk_groups=1, topk=2),
+                                dict(T=200, dim=256, moe_inter=128, n_routed=1024, n_groups=32,
+                                     topk_groups=8, topk=32)])
 def test_tensor_core_experts_match_oracle(kw, which):
     cfg = bf16_small(**kw)
     L, r, idx, w = _experts_case(cfg)
