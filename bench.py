@@ -349,7 +349,11 @@ def ours_arm(a, D):
     D.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    M.moe_stage_timing_begin(a.steps)
+    # per-kernel CUDA events on one step in `every` (about 20 steps), inside
+    # the same timed loop: events between every kernel of every step would
+    # cost the decode step ~1%
+    every = max(1, a.steps // 20)
+    M.moe_stage_timing_begin_every((a.steps + every - 1) // every, every)
     wall0 = time.time()
     ev0.record(stream)
     for _ in range(a.steps):
@@ -478,7 +482,8 @@ def ours_arm(a, D):
                                "frac_sustained": layer_roofline(
                                    cfg, n_active, dict(pk, bf16_tflops=pk["bf16_tflops_sustained"]))[2]
                                * 1e3 / ms_step},
-            "kernels_ms": per_kernel_ms, "dominant_kernel": dom, "active_experts": n_active,
+            "kernels_ms": per_kernel_ms, "kernels_ms_steps": {"recorded": n_rec, "every": every},
+            "dominant_kernel": dom, "active_experts": n_active,
             "routing": routing,
             "cpu_baseline": cpu, "clocks": ck,
         }

@@ -196,6 +196,12 @@ MOE_API moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void
 MOE_API moe_status moe_stage_timing_begin(int32_t max_calls);
 MOE_API int32_t moe_stage_timing_end(float* ms, int32_t n);
 
+/* moe_stage_timing_begin, recording only one moe_forward call in `every`
+ * (calls 0, every, 2*every, ... after arming), so that a timed loop carries
+ * the events of a few calls instead of all (each event recorded between two
+ * kernels costs the stream a little time). every >= 1. */
+MOE_API moe_status moe_stage_timing_begin_every(int32_t max_calls, int32_t every);
+
 /* Which kernels run the GEMMs of a bf16 layer, process-wide (for checks and
  * measurement; nothing switches on its own):
  *   AUTO (default)  tensor cores: router logits, and the grouped expert GEMM

@@ -35,7 +35,8 @@ MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch",
            "moe_experts_grouped", "moe_combine", "moe_forward", "moe_check_error",
            "moe_status_string", "moe_forward_launch_count", "moe_select_expert_kernel",
-           "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc")
+           "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc",
+           "moe_stage_timing_begin_every")
 
 # Kernels of moe_forward, in launch order.
 STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_scatter",
@@ -76,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward_launch_count": [C, I64],
         "moe_select_expert_kernel": [I32],
         "moe_stage_timing_begin": [I32],
+        "moe_stage_timing_begin_every": [I32, I32],
         "moe_stage_timing_end": [ctypes.POINTER(ctypes.c_float), I32],
         "moe_gate_noalloc": [C, I64, P, P, P, P, P, P],
     }
@@ -195,6 +197,11 @@ def moe_select_expert_kernel(which: int) -> None:
 
 def moe_stage_timing_begin(max_calls: int) -> None:
     _check(_lib.moe_stage_timing_begin(int(max_calls)), "moe_stage_timing_begin")
+
+
+def moe_stage_timing_begin_every(max_calls: int, every: int) -> None:
+    _check(_lib.moe_stage_timing_begin_every(int(max_calls), int(every)),
+           "moe_stage_timing_begin_every")
 
 
 def moe_stage_timing_end() -> tuple:

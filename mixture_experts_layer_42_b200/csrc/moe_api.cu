@@ -138,6 +138,8 @@ struct StageTiming {
   bool in_forward = false;
   int max_calls = 0;
   int calls = 0;          // moe_forward calls recorded
+  int every = 1;          // record one moe_forward call in `every`
+  int seen = 0;           // moe_forward calls since begin
   int marks = 0;          // events recorded in the current call
   int per_call = 0;       // events per call (kernels + 1)
   std::vector<cudaEvent_t> ev;
@@ -263,7 +265,8 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   cudaStream_t s = (cudaStream_t)stream;
   if ((st = bind_device(s, ws)) != MOE_OK) return st;
   StageTiming& TM = g_timing;
-  TM.in_forward = TM.on && TM.calls < TM.max_calls;
+  TM.in_forward = TM.on && TM.calls < TM.max_calls && TM.seen % TM.every == 0;
+  if (TM.on) ++TM.seen;
   if (TM.in_forward) {
     TM.marks = 0;
     stage_mark(s);
@@ -359,8 +362,11 @@ moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, con
 }
 
 moe_status moe_stage_timing_begin(int32_t max_calls) {
+  return moe_stage_timing_begin_every(max_calls, 1);
+}
+moe_status moe_stage_timing_begin_every(int32_t max_calls, int32_t every) {
   StageTiming& T = g_timing;
-  if (max_calls < 1 || max_calls > 4096) return MOE_ERR_INVALID_ARG;
+  if (max_calls < 1 || max_calls > 4096 || every < 1) return MOE_ERR_INVALID_ARG;
   for (cudaEvent_t e : T.ev) cudaEventDestroy(e);
   T.ev.clear();
   T.per_call = 2 + 3 + 2 + 1 + 1;
@@ -369,6 +375,8 @@ moe_status moe_stage_timing_begin(int32_t max_calls) {
     if (cudaEventCreate(&e) != cudaSuccess) return MOE_ERR_CUDA;
   T.max_calls = max_calls;
   T.calls = 0;
+  T.every = every;
+  T.seen = 0;
   T.on = true;
   return MOE_OK;
 }

@@ -357,3 +357,18 @@ def test_routing_profile_driver_runs(name, capsys):
     from mixture_experts_layer_42_b200 import profile_routing
     profile_routing.main(["--config", name, "--iters", "2"])
     assert "done" in capsys.readouterr().out
+
+
+def test_stage_timing_records_one_call_in_every():
+    L = Layer(bf16_small())
+    M.moe_stage_timing_begin_every(3, 2)       # calls 0, 2, 4 of the next seven
+    for _ in range(7):
+        L.forward()
+    n, ms = M.moe_stage_timing_end()
+    assert n == 3
+    assert all(v >= 0 for v in ms.values()) and ms["experts_up"] > 0
+    M.moe_stage_timing_begin(4)                # every call, up to four
+    for _ in range(5):
+        L.forward()
+    n, ms = M.moe_stage_timing_end()
+    assert n == 4 and ms["router_logits"] > 0
