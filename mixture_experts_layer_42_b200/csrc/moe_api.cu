@@ -68,19 +68,23 @@ int num_sms_current() {
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Make this thread's current device the one the caller's work lives on: the
-// stream's device, or for the legacy default stream the device of `ptr`.
+// device of `ptr` (a device buffer of the call), else the stream's device.
 // The library carries its own copy of the CUDA runtime, whose current device
-// does not follow the caller's runtime.
+// does not follow the caller's runtime. The pointer query comes first
+// because asking a stream for its device invalidates a CUDA graph capture
+// in progress on that stream, which would keep moe_forward out of graphs.
 moe_status bind_device(cudaStream_t s, const void* ptr) {
   int dev = -1;
-  if (s) {
-    if (cudaStreamGetDevice(s, &dev) != cudaSuccess) return MOE_ERR_CUDA;
-  } else {
+  if (ptr) {
     cudaPointerAttributes pa;
     if (cudaPointerGetAttributes(&pa, ptr) != cudaSuccess) return MOE_ERR_INVALID_ARG;
     if (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)
       return MOE_ERR_INVALID_ARG;
     dev = pa.device;
+  } else if (s) {
+    if (cudaStreamGetDevice(s, &dev) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    return MOE_ERR_INVALID_ARG;
   }
   int cur = -1;
   if (cudaGetDevice(&cur) != cudaSuccess) return MOE_ERR_CUDA;

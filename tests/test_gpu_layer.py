@@ -372,3 +372,37 @@ def test_stage_timing_records_one_call_in_every():
         L.forward()
     n, ms = M.moe_stage_timing_end()
     assert n == 4 and ms["router_logits"] > 0
+
+
+def test_forward_replays_from_a_cuda_graph():
+    # moe_forward does no host synchronisation and allocates nothing, so it can
+    # be captured once and replayed with new inputs written into the same buffers
+    cfg = bf16_small(T=300)
+    L = Layer(cfg)
+    ws = M.alloc_workspace(cfg, L.T)
+    y = torch.empty(L.T, cfg.dim, dtype=cfg.torch_dtype, device="cuda")
+    x = L.x.clone()
+    w1, w3, w2, ws1, ws3, ws2 = L.w
+    s = torch.cuda.Stream()
+
+    def run():
+        M.moe_forward(cfg, x, L.w_r, L.bias, w1, w3, w2, ws1, ws3, ws2, y, ws, stream=s)
+
+    with torch.cuda.stream(s):
+        run()                                   # warm-up outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run()
+    gen = torch.Generator().manual_seed(11)
+    for _ in range(3):
+        xi = torch.randn(L.T, cfg.dim, generator=gen).to(cfg.torch_dtype)
+        x.copy_(xi.cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        got = y.clone()
+        with torch.cuda.stream(s):
+            run()                               # the same inputs, eagerly
+        torch.cuda.synchronize()
+        assert torch.equal(got, y)
+        assert M.moe_check_error(ws) == M.MOE_OK
