@@ -31,9 +31,13 @@
  *     zeroed once by moe_workspace_init() after allocation. A workspace may be
  *     reused by any sequence of calls on one stream; calls that share a
  *     workspace must not run concurrently.
- *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call is
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream) of the device
+ *     that holds the call's workspace (moe_gate_noalloc: x). Every call is
  *     asynchronous on it and never synchronises the host, except
- *     moe_check_error.
+ *     moe_check_error. moe_gate, moe_dispatch, moe_experts_grouped,
+ *     moe_combine and moe_forward neither allocate, synchronise nor query
+ *     the stream, so they can be captured into a CUDA graph and replayed
+ *     with new data written into the same buffers.
  *   - Argument checks are synchronous: a bad config, size or pointer returns
  *     MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE before
  *     anything is launched. A failed launch returns MOE_ERR_CUDA.
