@@ -1,0 +1,61 @@
+"""The benchmark's command-line contract on the CPU: the reference arm (the
+CPU oracle timed on the host cores) prints exactly one JSON line with the
+keys the driver reads, alone and as two torchrun ranks of which rank 0 alone
+prints. The GPU arm's line is checked by running bench.py on a GPU."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _json_lines(out: str):
+    return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+
+
+def _check_reference_line(d, n_gpus):
+    assert d["impl"] == "reference"
+    assert d["metric"].startswith("MoE-layer tokens/sec")
+    assert d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["n_gpus"] == n_gpus and d["steps"] == 2 and d["warmup"] == 1
+    assert d["config"]["workload"] == "tiny_fp32"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny_fp32",
+                        "--steps", "2", "--warmup", "1"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 1)
+
+
+def test_reference_arm_under_torchrun_prints_on_rank_0_only():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+                        "--impl", "reference", "--gpus", "2", "--config", "tiny_fp32", "--steps", "2",
+                        "--warmup", "1"], cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    _check_reference_line(lines[0], 2)
+
+
+def test_gpu_count_must_match_the_launch():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--config",
+                        "tiny_fp32", "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode != 0 and "--gpus 2" in r.stderr
