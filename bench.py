@@ -249,8 +249,14 @@ def up_kernel_work(cfg, n_active):
 
 
 def source_digest(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 (16 hex digits) of a C++/CUDA source with its comments and
+    whitespace removed: it changes when the code changes, not the comments."""
+    import re
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return hashlib.sha256("".join(src.split()).encode()).hexdigest()[:16]
 
 
 def traffic_for(kernel, config_name):

@@ -20,6 +20,13 @@
 // (one 4D TMA box over both tensors when their distance allows, else two
 // boxes), so accumulator columns j and 128+j hold a and b of the same feature.
 //
+// An expert's last, partial m-tile loads its A rows through a copy of the A
+// tensor map whose row extent ends at the expert's last row (one per expert,
+// written by build_row_maps_kernel before the launch): TMA fills the rows
+// past it with zeros instead of the next expert's rows. The results are the
+// same (those rows are never stored), but zero operands draw less power, and
+// under the board's power cap that buys clock.
+//
 // Tiles are enumerated from the device offsets (no host round trip): expert
 // by expert, n-tile outer and m-tile inner so that CTAs running at the same
 // time share weight tiles and A rows in L2. Every pipeline wait is bounded
