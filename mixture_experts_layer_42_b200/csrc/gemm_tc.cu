@@ -60,6 +60,7 @@ struct Tile {
   int row0;   // first A row
   int rows;   // valid rows (<= BM)
   int n0;     // first output column
+  bool only;  // the expert's only m-tile
 };
 
 struct Sched {
@@ -86,6 +87,7 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
     t.row0 = S.off[e] + m * BM;
     t.rows = min(BM, S.off[e + 1] - t.row0);
     t.n0 = nt * S.bn_out;
+    t.only = mt == 1;
   } else {
     const int l = i - S.routed;
     const int nt = l / S.mt_sh, m = l % S.mt_sh;
@@ -94,9 +96,30 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
     t.row0 = m * BM;
     t.rows = min(BM, S.t_shared - t.row0);
     t.n0 = nt * S.bn_out;
+    t.only = false;
   }
   return t;
 }
+
+// The tile of an expert with at most SWAP_ROWS rows (its only tile; routed,
+// row maps built) runs with the operands swapped: the 128 weight rows of each
+// half of the B tile are the MMA's M side and the tile's r token rows,
+// rounded up to r16, its N side. The token box of that expert's row map is
+// r16 rows high, so the stage carries r16 token rows instead of 128, and the
+// MMAs do r16 columns of work instead of 128 padded rows. At decode batch
+// sizes (a few rows per expert) this removes most of the tensor work and its
+// power, and the SM clock rises under the power cap (2.33 -> 2.17 ms per V3
+// decode step). Experts with several m-tiles keep the plain form for their
+// last tile: their m-tiles stream the same weight tiles side by side and
+// share them in L2, which holds only while every m-tile runs at the same pace
+// (a swapped tile drifts out of step and re-reads its weights from HBM).
+// Single tiles of more than SWAP_ROWS rows also stay plain: swapping them
+// measured slower at prefill.
+constexpr int SWAP_ROWS = 64;
+__device__ __forceinline__ bool swap_tail(const Tile& t, const TcArgs& g) {
+  return t.kind == 0 && t.only && t.rows <= SWAP_ROWS && g.row_maps != nullptr;
+}
+__device__ __forceinline__ int tail_n(int rows) { return (rows + 15) & ~15; }
 
 __device__ __forceinline__ float silu_fast(float u) { return u / (1.0f + __expf(-u)); }
 
@@ -189,16 +212,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
         // an expert's last tile reads zeros past its rows, not the next
         // expert's (the padding rows then cost the tensor cores less power)
+        // an expert's last, partial tile reads zeros past its rows, not the
+        // next expert's; a swapped tile's box is only tail_n(rows) rows high
         const CUtensorMap* ta = &g.tmA[t.kind];
+        uint32_t tx = STAGE_BYTES;
         if (t.kind == 0 && t.rows < BM && g.row_maps != nullptr) {
           ta = g.row_maps + t.e;
           tmap_acquire(ta);
+          if (swap_tail(t, g)) tx = (uint32_t)(tail_n(t.rows) * BK * 2 + B_TILE);
         }
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err)) { ok = false; break; }
           uint8_t* sa = tiles + s * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
-          mbar_expect_tx(&full[s], STAGE_BYTES);
+          mbar_expect_tx(&full[s], tx);
           tma_load_2d(sa, ta, &full[s], kb * BK, t.row0);
           if (UP && g.b13[t.kind]) {
             tma_load_4d(sb, &g.tmB13[t.kind], &full[s], kb * BK, t.n0, t.e, 0);
@@ -234,14 +261,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
         if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, g.err)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        const bool swap = swap_tail(t, g);
+        // swapped tail: w1 (UP) or w2 rows 0-127 (DOWN) into TMEM columns
+        // [0, r16), w3 or w2 rows 128-255 into [128, 128 + r16)
+        const uint32_t idesc_t = idesc_bf16(BM, tail_n(t.rows));
+        const uint32_t w_lo = (UP && g.b13[t.kind] == 2) ? B_TILE / 2 : 0, w_hi = B_TILE / 2 - w_lo;
         for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(tiles + s * STAGE_BYTES);
           const uint32_t b0 = a0 + A_TILE;
+          if (swap) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint32_t acc_flag = (kb | kk) != 0 ? 1u : 0u;
+              tc_mma(d, sdesc(b0 + w_lo + kk * 32), sdesc(a0 + kk * 32), idesc_t, acc_flag);
+              tc_mma(d + BN / 2, sdesc(b0 + w_hi + kk * 32), sdesc(a0 + kk * 32), idesc_t, acc_flag);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc_mma(d, sdesc(a0 + kk * 32), sdesc(b0 + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[s]);
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
@@ -271,7 +312,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       const int n_out = g.n_out[t.kind];
       __nv_bfloat16* out =
           reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]) + (int64_t)(t.row0 + row) * n_out + t.n0;
-      if (UP) {
+      if (swap_tail(t, g)) {
+        // TMEM lane = output feature, column = token row of the tile
+        const int rn = tail_n(t.rows);
+        __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]) + (int64_t)t.row0 * n_out;
+        if (UP) {
+          const int f = t.n0 + row;            // this lane's feature
+#pragma unroll 1
+          for (int j = 0; j < rn; j += 16) {
+            uint32_t ra[16], rb[16];
+            tmem_ld16(tb + j, ra);
+            tmem_ld16(tb + BN / 2 + j, rb);
+            tmem_wait_ld();
+            if (f < n_out) {
+#pragma unroll
+              for (int q = 0; q < 16; ++q)
+                if (j + q < t.rows)
+                  base[(int64_t)(j + q) * n_out + f] = __float2bfloat16_rn(
+                      silu_fast(__uint_as_float(ra[q])) * __uint_as_float(rb[q]));
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            const int f = t.n0 + half * (BN / 2) + row;
+#pragma unroll 1
+            for (int j = 0; j < rn; j += 16) {
+              uint32_t ra[16];
+              tmem_ld16(tb + half * (BN / 2) + j, ra);
+              tmem_wait_ld();
+              if (f < n_out) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                  if (j + q < t.rows)
+                    base[(int64_t)(j + q) * n_out + f] = __float2bfloat16_rn(__uint_as_float(ra[q]));
+              }
+            }
+          }
+        }
+      } else if (UP) {
         // accumulator columns of w1 (a) and w3 (b): w3 first when its tile
         // came first in the paired load
         const uint32_t ca = g.b13[t.kind] == 2 ? BN / 2 : 0, cb = BN / 2 - ca;
@@ -346,10 +425,18 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
   __syncwarp();
   if (lane == 0) {
     const int end = offsets[e + 1];
+    // an expert with at most SWAP_ROWS rows: its only tile runs swapped, with
+    // a token box of tail_n(rows) rows; other experts keep BM-row boxes
+    const int tail = end - offsets[e] <= SWAP_ROWS ? end - offsets[e] : 0;
     asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], 1, %1;" ::"r"(
                      smem_u32(&sm[w])),
                  "r"(end > 0 ? end : 1)
                  : "memory");
+    if (tail > 0)
+      asm volatile("tensormap.replace.tile.box_dim.shared::cta.b1024.b32 [%0], 1, %1;" ::"r"(
+                       smem_u32(&sm[w])),
+                   "r"(tail_n(tail))
+                   : "memory");
   }
   __syncwarp();
   asm volatile(
