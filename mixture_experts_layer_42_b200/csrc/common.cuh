@@ -47,7 +47,8 @@ struct WsLayout {
   size_t s;             // [T, D] act
   size_t h;             // [T * k, I] act
   size_t hs;            // [T, I_s] act
-  size_t row_maps;      // [2, E] TMA maps (128 B): A rows of each expert (up, down)
+  size_t row_maps;      // [2, E] TMA maps (128 B): A rows of each expert (up, down),
+                        // then the tile counters of the up and down launches, 64 B apart
   size_t total;
   int router_splits;
   int n_chunks;
@@ -99,7 +100,7 @@ inline WsLayout ws_layout(const moe_config& c, int64_t T) {
   L.s = take((size_t)T * D * ab);
   L.h = take((size_t)T * k * I * ab);
   L.hs = take((size_t)T * (Is > 0 ? Is : 1) * ab);
-  L.row_maps = take((size_t)2 * E * 128);
+  L.row_maps = take((size_t)2 * E * 128 + 128);
   L.total = off;
   return L;
 }
@@ -201,7 +202,7 @@ enum { TC_ROWS = 0, TC_PAIR = 1 };
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
-                              void* out1, const int32_t* offsets, void* row_maps, uint32_t* err,
-                              int num_sms, cudaStream_t st);
+                              void* out1, const int32_t* offsets, void* row_maps, int* tile_ctr,
+                              uint32_t* err, int num_sms, cudaStream_t st);
 
 }  // namespace moe

@@ -50,6 +50,7 @@ constexpr int STAGE_BYTES = A_TILE + B_TILE;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_E = 1024;
+constexpr int TQ = 4;                      // tile queue depth (dynamic schedule)
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * (MAX_E + 1) * 4;
 
 constexpr uint32_t IDESC = tc::idesc_bf16(BM, BN);
@@ -115,6 +116,16 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
 // (a swapped tile drifts out of step and re-reads its weights from HBM).
 // Single tiles of more than SWAP_ROWS rows also stay plain: swapping them
 // measured slower at prefill.
+// Slot and phase parity of the shared-memory tile queue, kept by each role
+// that reads or writes it.
+struct TileQueue {
+  int q = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void advance() {
+    if (++q == TQ) { q = 0; ph ^= 1; }
+  }
+};
+
 constexpr int SWAP_ROWS = 64;
 __device__ __forceinline__ bool swap_tail(const Tile& t, const TcArgs& g) {
   return t.kind == 0 && t.only && t.rows <= SWAP_ROWS && g.row_maps != nullptr;
@@ -133,8 +144,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* qfull = drain + 1;            // tile queue: index written
+  uint64_t* qempty = qfull + TQ;          //             index read by the MMA and 4 epilogue warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + TQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* tq = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [TQ] tile indices
   int32_t* P = reinterpret_cast<int32_t*>(tiles + STAGES * STAGE_BYTES + 256);
   int32_t* off = P + MAX_E + 1;
 
@@ -145,6 +159,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     if (lane == 0) {
       for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
       for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+      for (int q = 0; q < TQ; ++q) { mbar_init(&qfull[q], 1); mbar_init(&qempty[q], 1 + 4); }
       mbar_init(drain, 1);
       *abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -207,11 +222,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       int s = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int i = blockIdx.x; ok && i < S.total; i += gridDim.x) {
+      TileQueue Q;
+      const bool dyn = g.tile_ctr != nullptr;
+      // the next tile is claimed a few k-blocks before the current one ends,
+      // so the atomic's round trip overlaps the current tile's loads
+      int next = dyn ? atomicAdd(g.tile_ctr, 1) : (int)blockIdx.x;
+      for (;;) {
+        const int i = next;
+        if (dyn) {
+          // hand the tile's index to the MMA and epilogue warps
+          if (!mbar_wait(&qempty[Q.q], Q.ph ^ 1, abort_flag, g.err)) { ok = false; break; }
+          tq[Q.q] = i;
+          mbar_arrive(&qfull[Q.q]);
+          Q.advance();
+        } else {
+          next = i + (int)gridDim.x;
+        }
+        if (i >= S.total) break;
         const Tile t = decode(S, i);
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
-        // an expert's last tile reads zeros past its rows, not the next
-        // expert's (the padding rows then cost the tensor cores less power)
+        const int kb_claim = kb_n > 4 ? kb_n - 4 : 0;
         // an expert's last, partial tile reads zeros past its rows, not the
         // next expert's; a swapped tile's box is only tail_n(rows) rows high
         const CUtensorMap* ta = &g.tmA[t.kind];
@@ -222,6 +252,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
           if (swap_tail(t, g)) tx = (uint32_t)(tail_n(t.rows) * BK * 2 + B_TILE);
         }
         for (int kb = 0; kb < kb_n; ++kb) {
+          if (dyn && kb == kb_claim) next = atomicAdd(g.tile_ctr, 1);
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err)) { ok = false; break; }
           uint8_t* sa = tiles + s * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
@@ -238,6 +269,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1; }
         }
+        if (!ok) break;
       }
       if (!ok) {
         // let every copy still in flight land before the CTA exits
@@ -250,10 +282,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int s = 0, lt = 0;
+      int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int i = blockIdx.x; ok && i < S.total; i += gridDim.x, ++lt) {
+      TileQueue Q;
+      for (int lt = 0; ok; ++lt) {
+        int i;
+        if (g.tile_ctr != nullptr) {
+          if (!mbar_wait(&qfull[Q.q], Q.ph, abort_flag, g.err)) break;
+          i = tq[Q.q];
+          mbar_arrive(&qempty[Q.q]);
+          Q.advance();
+        } else {
+          i = blockIdx.x + lt * gridDim.x;
+        }
+        if (i >= S.total) break;
         const Tile t = decode(S, i);
         const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
         const int acc = lt & 1;
@@ -297,8 +340,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     // ---------------------------------------------------------------- epilogue
     const int quad = warp & 3;           // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
-    int lt = 0;
-    for (int i = blockIdx.x; i < S.total; i += gridDim.x, ++lt) {
+    TileQueue Q;
+    for (int lt = 0;; ++lt) {
+      int i;
+      if (g.tile_ctr != nullptr) {
+        int w = 1;
+        i = 0;
+        if (lane == 0) {
+          w = mbar_wait(&qfull[Q.q], Q.ph, abort_flag, g.err) ? 1 : 0;
+          if (w) {
+            i = tq[Q.q];
+            mbar_arrive(&qempty[Q.q]);
+          }
+        }
+        w = __shfl_sync(0xffffffffu, w, 0);
+        i = __shfl_sync(0xffffffffu, i, 0);
+        if (!w) break;
+        Q.advance();
+      } else {
+        i = blockIdx.x + lt * gridDim.x;
+      }
+      if (i >= S.total) break;
       const Tile t = decode(S, i);
       const int acc = lt & 1;
       const uint32_t use = (uint32_t)(lt >> 1);
@@ -416,9 +478,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
 // publishes it to global memory with a release fence for the tensor-map proxy.
 __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ CUtensorMap base,
                                                              const int32_t* __restrict__ offsets,
-                                                             int E, CUtensorMap* maps) {
+                                                             int E, CUtensorMap* maps,
+                                                             int* tile_ctr) {
   __shared__ __align__(128) CUtensorMap sm[8];
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tile_ctr = 0;  // the GEMM's tile queue restarts
   const int e = blockIdx.x * 8 + w;
   if (e >= E) return;  // whole warps
   reinterpret_cast<uint32_t*>(&sm[w])[lane] = reinterpret_cast<const uint32_t*>(&base)[lane];
@@ -455,8 +519,8 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
-                              void* out1, const int32_t* offsets, void* row_maps, uint32_t* err,
-                              int num_sms, cudaStream_t st) {
+                              void* out1, const int32_t* offsets, void* row_maps, int* tile_ctr,
+                              uint32_t* err, int num_sms, cudaStream_t st) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
   const bool pair = kind == TC_PAIR;
@@ -530,10 +594,16 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
     stage_mark(st);
     return cudaSuccess;
   }
-  if (row_maps != nullptr && E > 0) {
+  if (row_maps != nullptr && tile_ctr != nullptr && E > 0) {
     g.row_maps = static_cast<const CUtensorMap*>(row_maps);
+    // Tiles in order from a counter for the up-projection: its long tiles
+    // (K = D) keep the CTAs that share weight and x_perm tiles in step, where
+    // round-robin lets them drift apart and re-read from HBM (UP read 1.15x
+    // its algorithmic DRAM bytes at prefill). The down-projection's tiles
+    // (K = I) are short enough that the hand-off costs more than it saves.
+    g.tile_ctr = up ? tile_ctr : nullptr;
     build_row_maps_kernel<<<(E + 7) / 8, 256, 0, st>>>(g.tmA[0], offsets, E,
-                                                       static_cast<CUtensorMap*>(row_maps));
+                                                       static_cast<CUtensorMap*>(row_maps), tile_ctr);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

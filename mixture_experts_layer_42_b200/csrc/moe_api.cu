@@ -104,14 +104,16 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
     // the same GPU, the pairs' 256-row tiles pad enough extra rows at the
     // DeepSeek-V3 prefill shape to lose to single CTAs under the power cap.
     const int kind = g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR ? TC_PAIR : TC_ROWS;
+    // tile counters of the up and down launches, after the 2 x E row maps
+    int* ctr = reinterpret_cast<int*>(static_cast<uint8_t*>(row_maps) + (size_t)2 * c.n_routed * 128);
     cudaError_t e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                                       c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
-                                      row_maps, err, num_sms_current(), st);
+                                      row_maps, ctr, err, num_sms_current(), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
                           c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets,
-                          static_cast<uint8_t*>(row_maps) + (size_t)c.n_routed * 128, err,
-                          num_sms_current(), st);
+                          static_cast<uint8_t*>(row_maps) + (size_t)c.n_routed * 128, ctr + 16,
+                          err, num_sms_current(), st);
     return cuda_status(e);
   }
   GroupedArgs g;

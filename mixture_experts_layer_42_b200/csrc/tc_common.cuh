@@ -274,6 +274,10 @@ struct TcArgs {
   // expert's last row (offsets[e + 1]), so that a tile reaching past it reads
   // zeros there; null when not built.
   const CUtensorMap* row_maps;
+  // One-CTA kernel: the launch's tile counter (zeroed by the row-map kernel
+  // before it); CTAs take tiles from it in order instead of round-robin by
+  // CTA index. Null: round-robin.
+  int* tile_ctr;
   int E;
   int t_shared;         // rows of the shared group (0: none)
   uint32_t* err;
