@@ -29,7 +29,11 @@
 //
 // Tiles are enumerated from the device offsets (no host round trip): expert
 // by expert, n-tile outer and m-tile inner so that CTAs running at the same
-// time share weight tiles and A rows in L2. Every pipeline wait is bounded
+// time share weight tiles and A rows in L2. The up-projection hands tiles out
+// in that order from a launch-wide counter (the TMA thread claims one and
+// passes its index to the MMA and epilogue warps through a small mbarrier
+// queue), which keeps the CTAs that share data starting together; the
+// down-projection assigns them round-robin by CTA. Every pipeline wait is bounded
 // (1 s); on expiry the kernel raises the timeout bit of the error word, drains
 // what it has in flight, frees TMEM and returns.
 #include "tc_common.cuh"
