@@ -106,6 +106,16 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
   return t;
 }
 
+// Slot and phase parity of the shared-memory tile queue, kept by each role
+// that reads or writes it.
+struct TileQueue {
+  int q = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void advance() {
+    if (++q == TQ) { q = 0; ph ^= 1; }
+  }
+};
+
 // The tile of an expert with at most SWAP_ROWS rows (its only tile; routed,
 // row maps built) runs with the operands swapped: the 128 weight rows of each
 // half of the B tile are the MMA's M side and the tile's r token rows,
@@ -120,16 +130,6 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
 // (a swapped tile drifts out of step and re-reads its weights from HBM).
 // Single tiles of more than SWAP_ROWS rows also stay plain: swapping them
 // measured slower at prefill.
-// Slot and phase parity of the shared-memory tile queue, kept by each role
-// that reads or writes it.
-struct TileQueue {
-  int q = 0;
-  uint32_t ph = 0;
-  __device__ __forceinline__ void advance() {
-    if (++q == TQ) { q = 0; ph ^= 1; }
-  }
-};
-
 constexpr int SWAP_ROWS = 64;
 __device__ __forceinline__ bool swap_tail(const Tile& t, const TcArgs& g) {
   return t.kind == 0 && t.only && t.rows <= SWAP_ROWS && g.row_maps != nullptr;
