@@ -224,6 +224,17 @@ enum {
 };
 MOE_API moe_status moe_select_expert_kernel(int32_t which);
 
+/* Test hook for the failure path of the tensor-core pipeline, process-wide,
+ * off by default; the pages have no counterpart. While enabled (1), the
+ * up-projection of every bf16 layer on the one-CTA tensor-core kernel has
+ * its first CTA wait, before it issues anything, on a barrier phase that
+ * nothing completes. The wait runs out after its 1 s limit; the launch then
+ * takes the abort path every timed-out wait takes (drain the copies in
+ * flight, free TMEM, return) and sets the timeout bit, so the next
+ * moe_check_error() returns MOE_ERR_TIMEOUT. The rows of that CTA's tiles are
+ * not written. 0 disables it; other values return MOE_ERR_INVALID_ARG. */
+MOE_API moe_status moe_debug_stall_pipeline(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch
            "moe_experts_grouped", "moe_combine", "moe_forward", "moe_check_error",
            "moe_status_string", "moe_forward_launch_count", "moe_select_expert_kernel",
            "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc",
-           "moe_stage_timing_begin_every")
+           "moe_stage_timing_begin_every", "moe_debug_stall_pipeline")
 
 # Kernels of moe_forward, in launch order.
 STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_scatter",
@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "moe_select_expert_kernel": [I32],
         "moe_stage_timing_begin": [I32],
         "moe_stage_timing_begin_every": [I32, I32],
+        "moe_debug_stall_pipeline": [I32],
         "moe_stage_timing_end": [ctypes.POINTER(ctypes.c_float), I32],
         "moe_gate_noalloc": [C, I64, P, P, P, P, P, P],
     }
@@ -189,6 +190,10 @@ def moe_check_error(ws, stream=None) -> int:
 
 def moe_forward_launch_count(cfg, T: int) -> int:
     return int(_lib.moe_forward_launch_count(_c(cfg), int(T)))
+
+
+def moe_debug_stall_pipeline(enable: int) -> None:
+    _check(_lib.moe_debug_stall_pipeline(int(enable)), "moe_debug_stall_pipeline")
 
 
 def moe_select_expert_kernel(which: int) -> None:

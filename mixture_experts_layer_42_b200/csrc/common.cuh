@@ -199,6 +199,9 @@ cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const G
                                 cudaStream_t st);
 // Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).
 enum { TC_ROWS = 0, TC_PAIR = 1 };
+// Test hook: the one-CTA up-projection's CTA 0 lets its first pipeline wait
+// run out (moe_debug_stall_pipeline).
+void set_pipeline_stall(bool on);
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,

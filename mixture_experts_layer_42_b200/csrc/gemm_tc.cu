@@ -290,6 +290,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       uint32_t ph = 0;
       bool ok = true;
       TileQueue Q;
+      // test hook: a wait that runs out (the drain barrier is committed only
+      // after the tile loop), before any MMA is issued
+      if (g.stall && blockIdx.x == 0 && !mbar_wait(drain, 0, abort_flag, g.err)) ok = false;
       for (int lt = 0; ok; ++lt) {
         int i;
         if (g.tile_ctr != nullptr) {
@@ -520,6 +523,10 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
 // and shared [N1, K1]; outputs [Tk, N0] and [T, N1]. `kind` picks the
 // kernel: TC_ROWS this one (128-row tiles), TC_PAIR the CTA-pair kernel
 // (256-row tiles, gemm_tc2.cu).
+// Test hook state (moe_debug_stall_pipeline).
+static bool g_stall = false;
+void set_pipeline_stall(bool on) { g_stall = on; }
+
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
@@ -606,6 +613,7 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
     // its algorithmic DRAM bytes at prefill). The down-projection's tiles
     // (K = I) are short enough that the hand-off costs more than it saves.
     g.tile_ctr = up ? tile_ctr : nullptr;
+    g.stall = up && g_stall ? 1 : 0;
     build_row_maps_kernel<<<(E + 7) / 8, 256, 0, st>>>(g.tmA[0], offsets, E,
                                                        static_cast<CUtensorMap*>(row_maps), tile_ctr);
     e = cudaGetLastError();

@@ -406,6 +406,12 @@ int32_t moe_stage_timing_end(float* ms, int32_t n) {
   return T.calls;
 }
 
+moe_status moe_debug_stall_pipeline(int32_t enable) {
+  if (enable != 0 && enable != 1) return MOE_ERR_INVALID_ARG;
+  set_pipeline_stall(enable != 0);
+  return MOE_OK;
+}
+
 moe_status moe_select_expert_kernel(int32_t which) {
   if (which != MOE_EXPERT_KERNEL_AUTO && which != MOE_EXPERT_KERNEL_SIMT &&
       which != MOE_EXPERT_KERNEL_TCGEN05 && which != MOE_EXPERT_KERNEL_TCGEN05_PAIR)

@@ -278,6 +278,10 @@ struct TcArgs {
   // before it); CTAs take tiles from it in order instead of round-robin by
   // CTA index. Null: round-robin.
   int* tile_ctr;
+  // Test hook (moe_debug_stall_pipeline): CTA 0's MMA thread first waits on
+  // a barrier phase that nothing completes, so that wait runs out (1 s)
+  // before anything is issued, and the launch takes its abort path.
+  int stall;
   int E;
   int t_shared;         // rows of the shared group (0: none)
   uint32_t* err;

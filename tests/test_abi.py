@@ -115,6 +115,11 @@ def test_workspace_size_grows_with_tokens(M):
     assert approx < ws < approx * 1.2
 
 
+def test_stall_hook_validates_its_argument(M):
+    assert M.raw_status("moe_debug_stall_pipeline", 2) == -1
+    assert M.raw_status("moe_debug_stall_pipeline", 0) == 0
+
+
 def test_launch_count(M):
     # bf16 on the one-CTA tensor-core kernel: each expert GEMM follows a
     # kernel that writes its per-expert A maps
