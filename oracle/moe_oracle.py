@@ -25,7 +25,7 @@ Sources (the pages this follows):
     SwiGLU, E(x) = w2 (silu(w1 x) * (w3 x)), silu(u) = u / (1 + e^-u), no
     biases, weights stored [out, in] like the router weight.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * ties in any top-k: the lower index wins; top-k output is ordered by
     descending score, then ascending index;
   * the accumulator is fp32 (the V3.2 page) and the shared expert is added
