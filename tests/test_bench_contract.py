@@ -1,6 +1,6 @@
 """The benchmark's command-line contract on the CPU: the reference arm (the
 CPU oracle timed on the host cores) prints exactly one JSON line with the
-keys the driver reads, alone and as two torchrun ranks of which rank 0 alone
+contract's keys, alone and as two torchrun ranks of which rank 0 alone
 prints. The GPU arm's line is checked by running bench.py on a GPU."""
 
 import json
