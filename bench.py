@@ -193,6 +193,15 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
+REFERENCE_BUDGET_S = 120.0   # wall time of the reference arm's warm-up and timed steps
+
+
+def host_bits(t):
+    """A tensor's values for the oracle: bf16 as raw uint16 bits, else numpy."""
+    t = t.detach().contiguous().cpu()
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+
 def oracle_rate(cfg, x_cpu, w_r, bias, w_dev, n_tok, seed=0, reps=1):
     """Tokens/s of the CPU oracle on a seeded sample of n_tok tokens of the
     workload (routing and experts of those tokens; a token's routing and
@@ -279,22 +288,47 @@ def traffic_for(kernel, config_name):
 # ---------------------------------------------------------------- arms
 
 def reference_arm(a, D):
-    """The CPU oracle, as it stands, on the host cores (rank 0 only)."""
+    """The CPU oracle, as it stands, on the host cores (rank 0 only). Every
+    step runs it on the same seeded token sample (the experts those tokens
+    use are copied to the host once, outside all timing); the sample is sized
+    from a one-token probe so that warm-up and timed steps together take
+    about REFERENCE_BUDGET_S seconds."""
     if D.rank != 0:
         return
+    from oracle import moe_oracle as O
     cfg = workload(a)
     x, w_r, bias = inputs.routing_inputs(cfg)
     w = inputs.expert_weights(cfg, "cuda" if torch.cuda.is_available() else "cpu")
-    n_tok = a.cpu_tokens or (8 if cfg.dim >= 4096 else 64)
+    kw = dict(n_groups=cfg.n_groups, topk_groups=cfg.topk_groups, topk=cfg.topk,
+              score_func=cfg.score, route_scale=cfg.route_scale)
+    xs_all, wr = host_bits(x), host_bits(w_r)
+    b = None if bias is None else bias.numpy().astype(np.float64)
+    rng = np.random.default_rng(1000)
+    cap = a.cpu_tokens or (8 if cfg.dim >= 4096 else 64)
+    tok = np.sort(rng.choice(x.shape[0], size=min(cap, x.shape[0]), replace=False))
+    r = O.route(O.router_logits(xs_all[tok], wr), b, **kw)
+    w1, w3, w2, ws1, ws3, ws2 = w
+    hw = {e: (host_bits(w1[e]), host_bits(w3[e]), host_bits(w2[e]))
+          for e in sorted(set(r["idx"].ravel().tolist()))}
+    shared = None if ws1 is None else (host_bits(ws1), host_bits(ws3), host_bits(ws2))
+
+    def run(n):
+        t0 = time.perf_counter()
+        O.moe_forward(xs_all[tok[:n]], wr, b, lambda e: hw[e], shared, act_dtype=cfg.dtype, **kw)
+        return time.perf_counter() - t0
+
+    t_one = run(1)
+    n_tok = int(max(1, min(len(tok), REFERENCE_BUDGET_S / max(t_one, 1e-6) / (a.warmup + a.steps))))
     rates = []
     for i in range(a.warmup + a.steps):
-        rate, n, n_used, _ = oracle_rate(cfg, x, w_r, bias, w, n_tok, seed=1000 + i)
+        dt = run(n_tok)
         if i >= a.warmup:
-            rates.append(rate)
+            rates.append(n_tok / dt)
     v = float(np.median(rates))
     cores = blas_threads()
-    sample = (f"{n_tok} seeded tokens of the {cfg.name} batch per step (their routing and "
-              f"experts, fp64 numpy oracle); median of {a.steps} steps")
+    sample = (f"the same {n_tok} seeded tokens of the {cfg.name} batch every step (their routing "
+              f"and experts, fp64 numpy oracle; sized to a ~{REFERENCE_BUDGET_S:.0f} s run); "
+              f"median of {a.steps} steps")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": cfg.T / v * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
