@@ -209,10 +209,7 @@ def oracle_rate(cfg, x_cpu, w_r, bias, w_dev, n_tok, seed=0, reps=1):
     outside the timed part."""
     from oracle import moe_oracle as O
 
-    def host(t):
-        t = t.detach().contiguous().cpu()
-        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
-
+    host = host_bits
     rng = np.random.default_rng(seed)
     tok = np.sort(rng.choice(x_cpu.shape[0], size=min(n_tok, x_cpu.shape[0]), replace=False))
     xs, wr = host(x_cpu)[tok], host(w_r)
