@@ -164,7 +164,10 @@ MOE_API moe_status moe_check_error(void* ws, void* stream);
 /* Static text for a status code. */
 MOE_API const char* moe_status_string(moe_status st);
 
-/* Number of kernels moe_forward launches for this config (for accounting). */
+/* Number of kernels moe_forward launches for this config with the expert
+ * kernel currently selected (moe_select_expert_kernel), for accounting: 10
+ * for a bf16 layer on the default one-CTA tensor-core kernel (each expert GEMM
+ * follows a kernel that writes its per-expert A maps), 8 otherwise. */
 MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
 
 /* moe_gate without a workspace. The pages have no counterpart of this call:
