@@ -59,3 +59,16 @@ def test_gpu_count_must_match_the_launch():
                         "tiny_fp32", "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode != 0 and "--gpus 2" in r.stderr
+
+
+def test_l2_note_states_how_the_timed_loop_meets_l2():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_42_b200 import inputs
+    big = bench.l2_note(inputs.CONFIGS["v3_decode"], 158)
+    assert big.startswith("inputs larger than L2") and "14.0 GB" in big   # 158 experts + shared
+    small = bench.l2_note(inputs.CONFIGS["tiny_fp32"], 16)
+    assert small.startswith("inputs fit in L2")
+    # the rest of the roofline inputs the GPU arm builds its line from
+    flops, byts, t, bound = bench.layer_roofline(inputs.CONFIGS["v3_decode"], 158, bench.NOMINAL_PEAKS)
+    assert bound == "hbm" and t > 0
