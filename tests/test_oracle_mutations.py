@@ -62,6 +62,23 @@ MUTATIONS = [
      [TR.test_round_bf16_matches_torch]),
     ("bf16 truncates", "np.round(m * 256.0) / 256.0", "np.trunc(m * 256.0) / 256.0",
      [TR.test_round_bf16_matches_torch]),
+    ("fp32 rounding skipped",
+     "return np.asarray(v, dtype=np.float64).astype(np.float32).astype(np.float64)",
+     "return np.asarray(v, dtype=np.float64)", [TR.test_round_f32_known_values]),
+    ("fp32 rounding to half precision", "astype(np.float32).astype(np.float64)",
+     "astype(np.float16).astype(np.float64)", [TR.test_round_f32_known_values]),
+    ("margin ignores the group gap",
+     "margin = np.minimum(margin, gs[:, topk_groups - 1] - gs[:, topk_groups])", "margin = margin",
+     [TR.test_golden_group_gap_decides_margin, TR.pin_brute_force_margins]),
+    ("margin reaches the (k+2)-th expert", "order[:, :min(topk + 1, E)]", "order[:, :min(topk + 2, E)]",
+     [TR.pin_brute_force_margins]),
+    ("margin skips the best expert left out", "order[:, :min(topk + 1, E)]", "order[:, :topk]",
+     [TR.test_golden_softmax, TR.pin_brute_force_margins]),
+    ("margin from unbiased scores", "ranked = np.take_along_axis(b, order", "ranked = np.take_along_axis(s, order",
+     [TR.test_golden_sigmoid_groups, TR.pin_brute_force_margins]),
+    ("group gap taken one group too deep", "gs[:, topk_groups - 1] - gs[:, topk_groups]",
+     "gs[:, topk_groups] - gs[:, min(topk_groups + 1, n_groups - 1)]",
+     [TR.test_golden_group_gap_decides_margin, TR.pin_brute_force_margins]),
 ]
 
 

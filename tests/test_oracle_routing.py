@@ -41,6 +41,33 @@ def test_round_bf16_matches_torch():
     np.testing.assert_array_equal(ours, ref)
 
 
+def test_round_f32_known_values():
+    # binary32 keeps 24 significant bits: 1 + 2^-23 is the next value after 1;
+    # halfway cases go to the even significand
+    u = 2.0 ** -23
+    cases = [
+        (1.0 + u / 2, 1.0),                          # halfway, 1.0 is even
+        (1.0 + 3 * u / 2, 1.0 + 2 * u),              # halfway, 1 + 2u is even
+        (1.0 + u / 2 + 2.0 ** -40, 1.0 + u),         # just above halfway rounds up
+        (1.0 + u / 2 - 2.0 ** -40, 1.0),             # just below rounds down
+        (-(1.0 + 3 * u / 2), -(1.0 + 2 * u)),        # symmetric in sign
+        (2.0 ** -149, 2.0 ** -149),                  # smallest subnormal is kept
+        (2.0 ** -150, 0.0),                          # halfway to 0, 0 is even
+        (3 * 2.0 ** -151, 2.0 ** -149),              # 0.75 of the smallest subnormal
+        (1.0 / 3.0, 11184811 * 2.0 ** -25),          # nearest binary32 to 1/3
+        (float(2 ** 24 + 1), float(2 ** 24)),        # integers past 2^24 lose the last bit
+    ]
+    v = np.array([c[0] for c in cases])
+    np.testing.assert_array_equal(O.round_f32(v), np.array([c[1] for c in cases]))
+
+
+def test_round_f32_matches_torch():
+    rng = np.random.default_rng(1)
+    v = rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000)
+    ref = torch.from_numpy(v).to(torch.float32).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_f32(v), ref)
+
+
 def test_to_f64_from_bf16_bits():
     v = torch.randn(1000, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
     bits = v.view(torch.int16).numpy().view(np.uint16)
@@ -49,8 +76,8 @@ def test_to_f64_from_bf16_bits():
 
 # ---------------------------------------------------------------- hand-worked examples
 
-def test_golden_sigmoid_groups():
-    g = _golden()["sigmoid_groups"]
+def _golden_sigmoid(name):
+    g = _golden()[name]
     s = np.array(g["s"])
     z = np.log(s / (1 - s))[None, :]
     # with x = z and W_r = identity the logits are z (page "Expert scores": z = x W_r)
@@ -60,6 +87,15 @@ def test_golden_sigmoid_groups():
     assert r["groups"][0].tolist() == g["expected_groups"]
     assert r["idx"][0].tolist() == g["expected_idx"]
     np.testing.assert_allclose(r["weights"][0], g["expected_weights"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["margin"][0], g["expected_margin"], rtol=0, atol=1e-12)
+
+
+def test_golden_sigmoid_groups():
+    _golden_sigmoid("sigmoid_groups")
+
+
+def test_golden_group_gap_decides_margin():
+    _golden_sigmoid("sigmoid_group_gap_decides")
 
 
 def test_golden_softmax():
@@ -68,6 +104,7 @@ def test_golden_softmax():
                score_func="softmax", route_scale=g["route_scale"])
     assert r["idx"][0].tolist() == g["expected_idx"]
     np.testing.assert_allclose(r["weights"][0], g["expected_weights"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["margin"][0], g["expected_margin"], rtol=0, atol=1e-12)
 
 
 def test_golden_dispatch():
@@ -114,7 +151,18 @@ def _brute_force(z, bias, n_groups, topk_groups, topk, score_func):
         elif tot > second:
             second = tot
     assert best_sum > second  # unique optimum on random inputs
-    return kept, set(best), s, b
+    # the decisive gaps, from the enumerated sets and no sorting: kept groups
+    # against dropped ones, chosen experts against eligible ones left out, and
+    # the closest pair among the chosen (which fixes their order)
+    gaps = []
+    if n_groups > 1 and topk_groups < n_groups:
+        gaps.append(min(gs[i] for i in kept) - max(gs[o] for o in range(n_groups) if o not in kept))
+    rest = [e for e in eligible if e not in best]
+    if rest:
+        gaps.append(min(b[e] for e in best) - max(b[e] for e in rest))
+    gaps += [abs(b[i] - b[j]) for i, j in itertools.combinations(best, 2)]
+    margin = min(gaps) if gaps else math.inf
+    return kept, set(best), s, b, margin
 
 
 CASES = [
@@ -139,8 +187,9 @@ def test_brute_force_routing(E, G, TG, k, score, has_bias):
     bias = rng.standard_normal(E) * 0.1 if has_bias else None
     r = _route(z, bias, n_groups=G, topk_groups=TG, topk=k, score_func=score, route_scale=1.7)
     for t in range(T):
-        kept, chosen, s, b = _brute_force(list(z[t]), None if bias is None else list(bias),
-                                          G, TG, k, score)
+        kept, chosen, s, b, margin = _brute_force(list(z[t]), None if bias is None else list(bias),
+                                                  G, TG, k, score)
+        assert math.isclose(r["margin"][t], margin, rel_tol=0, abs_tol=1e-12)
         if G > 1:
             assert r["groups"][t].tolist() == kept
         assert set(r["idx"][t].tolist()) == chosen
@@ -152,6 +201,67 @@ def test_brute_force_routing(E, G, TG, k, score, has_bias):
         if score == "sigmoid":
             wt = [v / sum(wt) for v in wt]
         np.testing.assert_allclose(r["weights"][t], np.array(wt) * 1.7, rtol=1e-12)
+
+
+@pytest.mark.parametrize("E,G,TG,k,score,has_bias", [c for c in CASES if c[5]])
+def test_margin_is_the_routing_decision_radius(E, G, TG, k, score, has_bias):
+    """Shifting every biased score by less than margin/4 (a group's top-2 sum
+    then moves by less than margin/2) leaves the brute-force routing
+    unchanged; pushing the deciding pair towards each other by a little more
+    than the margin changes it. The shifts go through the bias, one token at
+    a time."""
+    rng = np.random.default_rng(100 + E + k)
+    T = 10
+    z = rng.standard_normal((T, E)) * 1.5
+    bias = rng.standard_normal(E) * 0.1
+    kw = dict(n_groups=G, topk_groups=TG, topk=k, score_func=score, route_scale=1.0)
+    r = _route(z, bias, **kw)
+    per = E // G
+    for t in range(T):
+        m = r["margin"][t]
+        ref = _brute_force(list(z[t]), list(bias), G, TG, k, score)
+        for _ in range(3):
+            d = rng.uniform(-1, 1, E) * 0.249 * m
+            got = _brute_force(list(z[t]), list(bias + d), G, TG, k, score)
+            assert got[0] == ref[0] and got[1] == ref[1]
+            rt = _route(z[t:t + 1], bias + d, **kw)
+            assert rt["idx"][0].tolist() == r["idx"][t].tolist()
+        # the deciding pair, pushed across its gap
+        b = ref[3]
+        idx = r["idx"][t].tolist()
+        d = np.zeros(E)
+        pair_gaps = [(abs(b[i] - b[j]), i, j) for a, i in enumerate(idx) for j in idx[a + 1:]]
+        elig = [e for e in range(E) if G == 1 or e // per in set(ref[0])]
+        rest = [e for e in elig if e not in idx]
+        if rest:
+            worst = min(idx, key=lambda e: b[e])
+            best_out = max(rest, key=lambda e: b[e])
+            pair_gaps.append((b[worst] - b[best_out], worst, best_out))
+        gap, hi, lo = min(pair_gaps)
+        if gap <= m * (1 + 1e-9):
+            d[hi] -= 0.6 * gap
+            d[lo] += 0.6 * gap
+        else:
+            # the group gap decides: lower every member of the worst kept
+            # group and raise every member of the best dropped group
+            gs = {gi: sorted(b[gi * per:(gi + 1) * per], reverse=True) for gi in range(G)}
+            score_g = {gi: v[0] + v[1] for gi, v in gs.items()}
+            kg = min(ref[0], key=lambda gi: score_g[gi])
+            dg = max((gi for gi in range(G) if gi not in ref[0]), key=lambda gi: score_g[gi])
+            d[kg * per:(kg + 1) * per] -= 0.3 * m
+            d[dg * per:(dg + 1) * per] += 0.3 * m
+        rt = _route(z[t:t + 1], bias + d, **kw)
+        flipped = _brute_force(list(z[t]), list(bias + d), G, TG, k, score)
+        assert rt["idx"][0].tolist() != r["idx"][t].tolist()
+        assert (flipped[0], flipped[1]) != (ref[0], ref[1]) or \
+            sorted(idx, key=lambda e: -flipped[3][e]) != idx
+
+
+def pin_brute_force_margins():
+    """Every brute-force shape family in one call (used by the planted-mistake
+    tests, which call pins without arguments)."""
+    for case in CASES:
+        test_brute_force_routing(*case)
 
 
 # ---------------------------------------------------------------- invariants
