@@ -256,6 +256,77 @@ def moe_layer(x: np.ndarray, weights: np.ndarray, idx: np.ndarray, experts, shar
     return round_to(y, act_dtype)
 
 
+# --------------------------------------------------------------------------
+# Expert parallelism (the MoE class on the hackaday page and DeepseekV3MoE on
+# the thataiguy page: rank r of world_size holds the contiguous block of
+# n_routed / world_size experts starting at r * n_routed / world_size; every
+# rank routes all tokens, runs only its own experts, and the ranks' partial
+# outputs are summed by one all_reduce of y. The V3.2 listing ("Weighted
+# expert sum", MoE.forward) adds the shared MLP into y before that all_reduce,
+# so each rank holds a slice of the shared MLP -- a block of its inner width
+# -- whose outputs add up to the whole MLP.)
+
+
+def expert_block(n_experts: int, world_size: int, rank: int) -> range:
+    """Experts held by `rank`: a contiguous block of n_experts / world_size."""
+    if n_experts % world_size:
+        raise ValueError("n_routed_experts must divide by world_size")
+    per = n_experts // world_size
+    return range(rank * per, (rank + 1) * per)
+
+
+def shared_block(shared_inter: int, world_size: int, rank: int) -> range:
+    """Inner features of the shared MLP held by `rank` (a contiguous block)."""
+    if shared_inter % world_size:
+        raise ValueError("the shared MLP's width must divide by world_size")
+    per = shared_inter // world_size
+    return range(rank * per, (rank + 1) * per)
+
+
+def moe_layer_partial(x: np.ndarray, weights: np.ndarray, idx: np.ndarray, experts, shared,
+                      *, expert_range: range, shared_range: range, act_dtype=None,
+                      tokens=None) -> np.ndarray:
+    """One rank's contribution to y before the all_reduce, in fp64 (not
+    rounded at the end): the weighted outputs of the experts in
+    `expert_range` for the tokens routed to them, plus the shared MLP
+    restricted to the inner features `shared_range` (rows of ws1 and ws3,
+    columns of ws2). Each expert's output and the shared slice's output are
+    rounded to `act_dtype` as in moe_layer."""
+    x = to_f64(x)
+    T, D = x.shape
+    rows = np.arange(T) if tokens is None else np.asarray(tokens)
+    xs, ws, ids = x[rows], np.asarray(weights, np.float64)[rows], np.asarray(idx)[rows]
+    y = np.zeros((len(rows), D))
+    for e in np.unique(ids):
+        if int(e) not in expert_range:
+            continue
+        r, j = np.nonzero(ids == e)
+        w1, w3, w2 = experts(int(e))
+        out = swiglu(xs[r], w1, w3, w2, round_h=act_dtype, round_out=act_dtype)
+        y[r] = y[r] + out * ws[r, j][:, None]
+    if shared is not None and len(shared_range):
+        ws1, ws3, ws2 = shared
+        f = np.asarray(shared_range)
+        y += swiglu(xs, np.asarray(ws1)[f], np.asarray(ws3)[f], np.asarray(ws2)[:, f],
+                    round_h=act_dtype, round_out=act_dtype)
+    return y
+
+
+def moe_layer_ep(x, weights, idx, experts, shared, *, n_experts, world_size, act_dtype=None,
+                 tokens=None) -> np.ndarray:
+    """The layer over `world_size` expert-parallel ranks: every rank's
+    partial output (its expert block and its slice of the shared MLP),
+    summed as the all_reduce does, then rounded once to `act_dtype`."""
+    Is = 0 if shared is None else np.asarray(shared[0]).shape[0]
+    y = 0.0
+    for r in range(world_size):
+        y = y + moe_layer_partial(x, weights, idx, experts, shared,
+                                  expert_range=expert_block(n_experts, world_size, r),
+                                  shared_range=shared_block(Is, world_size, r) if Is else range(0),
+                                  act_dtype=act_dtype, tokens=tokens)
+    return round_to(y, act_dtype)
+
+
 def moe_forward(x, w_router, bias, experts, shared, *, n_groups, topk_groups, topk,
                 score_func, route_scale, act_dtype=None, tokens=None) -> dict:
     """The whole layer: route every token, then combine (for `tokens`)."""

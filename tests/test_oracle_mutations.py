@@ -12,6 +12,7 @@ import types
 import pytest
 
 from oracle import moe_oracle
+from tests import test_oracle_ep as TEP
 from tests import test_oracle_experts as TE
 from tests import test_oracle_routing as TR
 
@@ -76,6 +77,15 @@ MUTATIONS = [
      [TR.test_golden_softmax, TR.pin_brute_force_margins]),
     ("margin from unbiased scores", "ranked = np.take_along_axis(b, order", "ranked = np.take_along_axis(s, order",
      [TR.test_golden_sigmoid_groups, TR.pin_brute_force_margins]),
+    ("expert block drops its last expert",
+     "per = n_experts // world_size\n    return range(rank * per, (rank + 1) * per)",
+     "per = n_experts // world_size\n    return range(rank * per, (rank + 1) * per - 1)",
+     [TEP.pin_ep_partials]),
+    ("every rank adds the whole shared MLP",
+     "y += swiglu(xs, np.asarray(ws1)[f], np.asarray(ws3)[f], np.asarray(ws2)[:, f],",
+     "y += swiglu(xs, np.asarray(ws1), np.asarray(ws3), np.asarray(ws2),", [TEP.pin_ep_partials]),
+    ("shared slice takes rows of ws2", "np.asarray(ws2)[:, f]", "np.asarray(ws2)[f, :].T",
+     [TEP.pin_ep_partials]),
     ("group gap taken one group too deep", "gs[:, topk_groups - 1] - gs[:, topk_groups]",
      "gs[:, topk_groups] - gs[:, min(topk_groups + 1, n_groups - 1)]",
      [TR.test_golden_group_gap_decides_margin, TR.pin_brute_force_margins]),
