@@ -83,6 +83,85 @@ def round_to(v: np.ndarray, dtype) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# FP8 (e4m3) block-scaled numbers. The pages say only that the block's other
+# linears are FP8 ("Expert scores", dtype note); the layout here is this
+# library's: e4m3 values (1 sign, 4 exponent bits with bias 7, 3 mantissa
+# bits, largest finite 448, subnormals down to 2^-9) with one power-of-two
+# scale per block -- 128 x 128 for a weight matrix [out, in], 1 x 128 for a row
+# of activations. A block's scale 2^s is the smallest with amax <= 448 * 2^s,
+# and its values are q = e4m3(v / 2^s) rounded to nearest, ties to even.
+
+E4M3_MAX = 448.0
+
+
+def round_e4m3(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest e4m3 value, ties to even, returned
+    as float64 (|v| <= 448 expected; larger magnitudes saturate to 448).
+    Normal range: v = m * 2^e with 0.5 <= |m| < 1 keeps m to 1/16; below
+    2^-6 the spacing is the subnormal step 2^-9."""
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)
+    normal = np.ldexp(np.round(m * 16.0) / 16.0, e)
+    sub = np.round(v * 512.0) / 512.0
+    out = np.where(np.abs(v) < 2.0 ** -6, sub, normal)
+    return np.clip(out, -E4M3_MAX, E4M3_MAX)
+
+
+def block_exponent(amax: np.ndarray) -> np.ndarray:
+    """Smallest integer s with amax <= 448 * 2^s (0 for an all-zero block)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    m, e = np.frexp(np.where(amax > 0, amax, 1.0))   # amax = m 2^e, 0.5 <= m < 1
+    # amax = (2m) 2^(e-1) and 448 = 1.75 * 2^8: s = e - 9, one more when 2m > 1.75
+    s = e - 9 + (2.0 * m > 1.75)
+    return np.where(amax > 0, s, 0).astype(np.int64)
+
+
+def quantize_blocks(a: np.ndarray, block_rows: int, block_cols: int):
+    """Quantize a 2D array to e4m3 with one power-of-two scale per block
+    (blocks of block_rows x block_cols, partial at the edges). Returns
+    (q [R, C] float64 e4m3 values, scale [ceil(R/br), ceil(C/bc)] powers of two)."""
+    a = to_f64(a)
+    R, C = a.shape
+    nr, nc = -(-R // block_rows), -(-C // block_cols)
+    q = np.empty_like(a)
+    scale = np.empty((nr, nc))
+    for i in range(nr):
+        for j in range(nc):
+            blk = a[i * block_rows:(i + 1) * block_rows, j * block_cols:(j + 1) * block_cols]
+            s = float(np.ldexp(1.0, int(block_exponent(np.abs(blk).max()))))
+            scale[i, j] = s
+            q[i * block_rows:(i + 1) * block_rows, j * block_cols:(j + 1) * block_cols] = \
+                round_e4m3(blk / s)
+    return q, scale
+
+
+def dequantize_blocks(q: np.ndarray, scale: np.ndarray, block_rows: int, block_cols: int):
+    """q * the scale of its block."""
+    q = np.asarray(q, dtype=np.float64)
+    full = np.repeat(np.repeat(np.asarray(scale, np.float64), block_rows, 0), block_cols, 1)
+    return q * full[:q.shape[0], :q.shape[1]]
+
+
+def fp8_act(a: np.ndarray) -> np.ndarray:
+    """Activations as the FP8 experts see them: quantized per 1 x 128 block
+    and dequantized."""
+    q, s = quantize_blocks(a, 1, 128)
+    return dequantize_blocks(q, s, 1, 128)
+
+
+def swiglu_fp8(xr, w1, w3, w2, round_out=None) -> np.ndarray:
+    """E(x) with FP8 block-scaled weights (given dequantized, [out, in]) and
+    FP8 activations: x and h are each quantized per 1 x 128 block before
+    their product; the products accumulate exactly (fp64 here); the output is
+    rounded to `round_out`."""
+    xq = fp8_act(xr)
+    a = xq @ to_f64(w1).T
+    c = xq @ to_f64(w3).T
+    h = fp8_act(silu(a) * c)
+    return round_to(np.matmul(h, to_f64(w2).T), round_out)
+
+
+# --------------------------------------------------------------------------
 # Step 1: router logits and scores ("Expert scores": z = x W_r, applied in
 # float32 -- here float64, which is the exact value up to rounding)
 
@@ -230,7 +309,7 @@ def swiglu(xr: np.ndarray, w1: np.ndarray, w3: np.ndarray, w2: np.ndarray,
 
 
 def moe_layer(x: np.ndarray, weights: np.ndarray, idx: np.ndarray, experts, shared,
-              *, act_dtype=None, tokens=None) -> np.ndarray:
+              *, act_dtype=None, tokens=None, fp8=False) -> np.ndarray:
     """y[t] = sum_j weights[t, j] * E_{idx[t, j]}(x[t]) + S(x[t]).
 
     `experts(e)` returns (w1, w3, w2) of routed expert e; `shared` is
@@ -239,6 +318,8 @@ def moe_layer(x: np.ndarray, weights: np.ndarray, idx: np.ndarray, experts, shar
     added and the sum is rounded once to `act_dtype` (None keeps fp64).
     `tokens` restricts the computation to a subset of token rows (a token's
     output depends only on its own row); the result then has len(tokens) rows.
+    With `fp8`, the expert weights are FP8 block-scaled (given dequantized)
+    and every expert, the shared MLP included, runs as swiglu_fp8.
     """
     x = to_f64(x)
     T, D = x.shape
@@ -248,11 +329,17 @@ def moe_layer(x: np.ndarray, weights: np.ndarray, idx: np.ndarray, experts, shar
     for e in np.unique(ids):
         r, j = np.nonzero(ids == e)                 # row-major, as where() gives
         w1, w3, w2 = experts(int(e))
-        out = swiglu(xs[r], w1, w3, w2, round_h=act_dtype, round_out=act_dtype)
+        if fp8:
+            out = swiglu_fp8(xs[r], w1, w3, w2, round_out=act_dtype)
+        else:
+            out = swiglu(xs[r], w1, w3, w2, round_h=act_dtype, round_out=act_dtype)
         y[r] += out * ws[r, j][:, None]
     if shared is not None:
         ws1, ws3, ws2 = shared
-        y += swiglu(xs, ws1, ws3, ws2, round_h=act_dtype, round_out=act_dtype)
+        if fp8:
+            y += swiglu_fp8(xs, ws1, ws3, ws2, round_out=act_dtype)
+        else:
+            y += swiglu(xs, ws1, ws3, ws2, round_h=act_dtype, round_out=act_dtype)
     return round_to(y, act_dtype)
 
 

@@ -14,6 +14,7 @@ import pytest
 from oracle import moe_oracle
 from tests import test_oracle_ep as TEP
 from tests import test_oracle_experts as TE
+from tests import test_oracle_fp8 as TF8
 from tests import test_oracle_routing as TR
 
 SRC = inspect.getsource(moe_oracle)
@@ -86,6 +87,17 @@ MUTATIONS = [
      "y += swiglu(xs, np.asarray(ws1), np.asarray(ws3), np.asarray(ws2),", [TEP.pin_ep_partials]),
     ("shared slice takes rows of ws2", "np.asarray(ws2)[:, f]", "np.asarray(ws2)[f, :].T",
      [TEP.pin_ep_partials]),
+    ("e4m3 keeps 4 mantissa bits", "normal = np.ldexp(np.round(m * 16.0) / 16.0, e)",
+     "normal = np.ldexp(np.round(m * 32.0) / 32.0, e)", [TF8.pin_fp8]),
+    ("e4m3 subnormal step 2^-8", "sub = np.round(v * 512.0) / 512.0", "sub = np.round(v * 256.0) / 256.0",
+     [TF8.pin_fp8]),
+    ("fp8 scale one step too large", "s = e - 9 + (2.0 * m > 1.75)", "s = e - 8 + (2.0 * m > 1.75)",
+     [TF8.pin_fp8]),
+    ("fp8 scale ignores the 1.75 boundary", "s = e - 9 + (2.0 * m > 1.75)", "s = e - 9 + (2.0 * m > 1.5)",
+     [TF8.pin_fp8]),
+    ("h not quantized before w2", "h = fp8_act(silu(a) * c)", "h = silu(a) * c", [TF8.pin_fp8]),
+    ("activations quantized per 128 x 128", "q, s = quantize_blocks(a, 1, 128)",
+     "q, s = quantize_blocks(a, 128, 128)", [TF8.pin_fp8]),
     ("group gap taken one group too deep", "gs[:, topk_groups - 1] - gs[:, topk_groups]",
      "gs[:, topk_groups] - gs[:, min(topk_groups + 1, n_groups - 1)]",
      [TR.test_golden_group_gap_decides_margin, TR.pin_brute_force_margins]),
