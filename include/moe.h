@@ -121,8 +121,10 @@ MOE_API moe_status moe_gate(const moe_config* cfg, int64_t T, const void* x, con
  * offsets[E] = number of valid pairs), src [T*k] (token of each permuted
  * row), pos [T*k] (permuted row of pair (t, j), -1 for an invalid index), and
  * x_perm [T*k, D] (act), x's rows in expert-contiguous order, ascending token
- * within an expert. An index outside [0, E) sets MOE_ERR_DEVICE_CHECK in the
- * error word and its pair is dropped. */
+ * within an expert. x_perm may be NULL (and x with it): then only counts,
+ * offsets, src and pos are written, for moe_experts_grouped_gather, which
+ * reads x's rows through src. An index outside [0, E) sets
+ * MOE_ERR_DEVICE_CHECK in the error word and its pair is dropped. */
 MOE_API moe_status moe_dispatch(const moe_config* cfg, int64_t T, const int32_t* idx, const void* x,
                         int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                         void* x_perm, void* ws, size_t ws_bytes, void* stream);
@@ -140,6 +142,20 @@ MOE_API moe_status moe_experts_grouped(const moe_config* cfg, int64_t T, const v
                                const void* ws3, const void* ws2, void* y_perm, void* s,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* moe_experts_grouped without the expert-contiguous copy of x: row p of the
+ * expert order is token src[p] of x [T, D] (src and offsets as moe_dispatch
+ * writes them), read straight from x by the expert GEMM (TMA gather of four
+ * token rows per copy on the tensor-core path). Same outputs as
+ * moe_experts_grouped on x_perm; x is required. This is how moe_forward runs
+ * the experts. Returns MOE_ERR_UNSUPPORTED for a bf16 layer while the
+ * CTA-pair expert kernel is selected (it reads only x_perm). */
+MOE_API moe_status moe_experts_grouped_gather(const moe_config* cfg, int64_t T, const void* x,
+                                              const int32_t* src, const int32_t* offsets,
+                                              const void* w1, const void* w3, const void* w2,
+                                              const void* ws1, const void* ws3, const void* ws2,
+                                              void* y_perm, void* s, void* ws, size_t ws_bytes,
+                                              void* stream);
+
 /* Combine (page "Weighted expert sum": y_routed = sum_i G_i E_i, accumulated
  * in float32 and cast back at the end; then the shared expert added):
  * y[t] = act( sum_j weights[t,j] * y_perm[pos[t,j]] + s[t] ), fp32 sum over
@@ -150,12 +166,106 @@ MOE_API moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_p
 
 /* The whole layer (MoE.forward): gate, dispatch, experts and combine chained
  * on `stream` with no host synchronisation. y [T, D] (act). weights_out
- * [T, k] and idx_out [T, k] may be NULL; when given they receive the routing. */
+ * [T, k] and idx_out [T, k] may be NULL; when given they receive the routing.
+ * For batches of at most 64 routed rows per expert on average (T * k <=
+ * 64 * n_routed: decode) and for fp32 layers, the experts read the routed
+ * token rows straight from x (as moe_experts_grouped_gather does) and no
+ * permuted copy of x is made. Larger bf16 batches, and the CTA-pair expert
+ * kernel, read an expert-contiguous copy that dispatch writes into the
+ * workspace's y_perm region (free until the down-projection writes it): on
+ * B200 the copy is the faster of the two for 128-row tiles. */
 MOE_API moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
                        const float* bias, const void* w1, const void* w3, const void* w2,
                        const void* ws1, const void* ws3, const void* ws2, void* y,
                        float* weights_out, int32_t* idx_out, void* ws, size_t ws_bytes,
                        void* stream);
+
+/* Expert parallelism (the MoE class on the hackaday page and DeepseekV3MoE on
+ * the thataiguy page: rank r of world_size holds the contiguous block of
+ * experts [r E / world_size, (r + 1) E / world_size); every rank routes all
+ * tokens and runs only its own experts, and one all_reduce sums the ranks'
+ * outputs. The V3.2 listing on page "Weighted expert sum" adds the shared MLP
+ * into y before that all_reduce, so each rank also holds a slice of the
+ * shared MLP's inner width; the slices' outputs add up to the whole MLP.)
+ *
+ * One rank's share of the layer: the gate over all E experts (W_r and bias
+ * whole), dispatch, the grouped experts for this rank's block [expert_begin,
+ * expert_end) only, and its shared slice, combined into y_partial [T, D]
+ * fp32 -- sum_j w[t,j] E_{idx[t,j]}(x[t]) over the pairs routed into the
+ * block, plus the slice's output -- not rounded. w1, w3 [n_local, I, D] and
+ * w2 [n_local, D, I] hold the block's experts (n_local = expert_end -
+ * expert_begin, first expert first); ws1, ws3 [shared_local, D] and ws2
+ * [D, shared_local] the rank's slice of the shared MLP (contiguous copies of
+ * rows of ws1 / ws3 and columns of ws2; NULL when shared_local == 0). The
+ * caller sums y_partial over the ranks in fp32 (an all_reduce) and casts the
+ * sum once with moe_cast_output. Workspace as for moe_forward. Requires
+ * 0 <= expert_begin < expert_end <= n_routed and 0 <= shared_local <=
+ * shared_inter (a multiple of 8 for bf16, 4 for fp32); MOE_ERR_UNSUPPORTED
+ * for a bf16 layer while the CTA-pair expert kernel is selected. */
+MOE_API moe_status moe_forward_ep(const moe_config* cfg, int64_t T, int32_t expert_begin,
+                                  int32_t expert_end, int32_t shared_local, const void* x,
+                                  const void* w_router, const float* bias, const void* w1,
+                                  const void* w3, const void* w2, const void* ws1, const void* ws3,
+                                  const void* ws2, float* y_partial, float* weights_out,
+                                  int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/* y [T, D] (act) = y_sum [T, D] (fp32) rounded once: the last step of an
+ * expert-parallel layer, after the ranks' y_partial have been summed. */
+MOE_API moe_status moe_cast_output(const moe_config* cfg, int64_t T, const float* y_sum, void* y,
+                                   void* stream);
+
+/* FP8 expert weights. The page "DeepSeek-V3.2-Exp - Expert scores" says the
+ * block's other linears are FP8 and gives no layout; this library's layout:
+ * e4m3 values (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; finite
+ * values up to 448), one fp32 scale per 128 x 128 block of each [out, in]
+ * matrix, a power of two: the smallest 2^s with the block's largest magnitude
+ * <= 448 * 2^s. A weight is q * scale. moe_quantize_fp8 produces the layout
+ * from bf16 or fp32 weights. Scales are row-major over the blocks:
+ * w1_scale / w3_scale [E, I/128, D/128], w2_scale [E, D/128, I/128],
+ * ws1_scale / ws3_scale [I_s/128, D/128], ws2_scale [D/128, I_s/128]. */
+typedef struct {
+  const void* w1;           /* e4m3 [E, I, D] */
+  const void* w3;           /* e4m3 [E, I, D] */
+  const void* w2;           /* e4m3 [E, D, I] */
+  const float* w1_scale;
+  const float* w3_scale;
+  const float* w2_scale;
+  const void* ws1;          /* shared MLP, e4m3 [I_s, D]; NULL when shared_inter == 0 */
+  const void* ws3;          /* e4m3 [I_s, D] */
+  const void* ws2;          /* e4m3 [D, I_s] */
+  const float* ws1_scale;
+  const float* ws3_scale;
+  const float* ws2_scale;
+} moe_fp8_weights;
+
+/* Quantize a [rows, cols] matrix a (the config's activation dtype) to e4m3
+ * with one power-of-two scale per block_rows x 128 block (block_rows = 128
+ * for weights, 1 for rows of activations): scales [ceil(rows/block_rows),
+ * cols/128] fp32, q [rows, cols] e4m3 bytes. Each value is rounded to the
+ * nearest e4m3 value, ties to even. cols must be a multiple of 128. Stacked
+ * expert weights [E, N, K] quantize as [E*N, K] when N is a multiple of 128. */
+MOE_API moe_status moe_quantize_fp8(const moe_config* cfg, const void* a, int64_t rows,
+                                    int64_t cols, int32_t block_rows, void* q, float* scales,
+                                    void* stream);
+
+/* Bytes of workspace moe_forward_fp8 needs for T tokens; MOE_ERR_UNSUPPORTED
+ * unless the layer is bf16 with dim, moe_inter and shared_inter multiples of
+ * 128 and at most 8192. */
+MOE_API moe_status moe_workspace_size_fp8(const moe_config* cfg, int64_t T, size_t* bytes);
+
+/* The whole layer with FP8 expert weights: the router as in moe_forward (bf16
+ * W_r applied in fp32), then x quantized per 1 x 128 block of each row to
+ * e4m3 (as the weights, one power-of-two scale per block), the routed and
+ * shared SwiGLU experts on the e4m3 tensor cores (kind::f8f6f4, fp32
+ * accumulation in 128-deep blocks scaled by the product of the weight's and
+ * the row's block scales), h = silu(w1 x) * (w3 x) quantized the same way
+ * before w2, each expert's output rounded to bf16, and the combine as in
+ * moe_forward. Workspace of moe_workspace_size_fp8() bytes, initialised by
+ * moe_workspace_init(). bf16 layers only. */
+MOE_API moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x,
+                                   const void* w_router, const float* bias,
+                                   const moe_fp8_weights* w, void* y, float* weights_out,
+                                   int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read and clear the workspace's error word. Returns
  * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT (or MOE_ERR_CUDA). */
@@ -165,9 +275,9 @@ MOE_API moe_status moe_check_error(void* ws, void* stream);
 MOE_API const char* moe_status_string(moe_status st);
 
 /* Number of kernels moe_forward launches for this config with the expert
- * kernel currently selected (moe_select_expert_kernel), for accounting: 10
- * for a bf16 layer on the default one-CTA tensor-core kernel (each expert GEMM
- * follows a kernel that writes its per-expert A maps), 8 otherwise. */
+ * kernel currently selected (moe_select_expert_kernel), for accounting: 9
+ * for a bf16 layer on the default one-CTA tensor-core kernel (the expert GEMMs
+ * follow one kernel that writes their per-expert A maps), 8 otherwise. */
 MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
 
 /* moe_gate without a workspace. The pages have no counterpart of this call:
@@ -180,15 +290,31 @@ MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
  * (1,048,576 floats; every GPU that loads the library holds it until the
  * process exits). Limit: T * n_routed <= 1,048,576 (T <= 4096 at 256
  * experts); larger shapes return MOE_ERR_UNSUPPORTED and launch nothing. The
- * call allocates no device memory. The first call on each device looks up the
- * scratch's device address (cudaGetSymbolAddress) and caches it. All calls
- * share the one array and it keeps the last call's partial sums (each call
- * overwrites every element it reads); calls whose work overlaps on the GPU,
- * on different streams or host threads, race on it and must be serialised
- * by the caller. */
+ * call allocates no device memory itself. The first call on each device looks
+ * up the scratch's device address (cudaGetSymbolAddress) and caches it; under
+ * CUDA's lazy module loading (the default) that first call may also be what
+ * loads the library's device code onto the device, which reserves the array
+ * and can synchronise. A latency-critical loop should therefore make one call
+ * (or one moe_gate_noalloc_check_error) on each device before it starts, and
+ * before any stream capture. All calls share the one array and it keeps the
+ * last call's partial sums (each call overwrites every element it reads);
+ * calls whose work overlaps on the GPU, on different streams or host threads,
+ * race on it and must be serialised by the caller.
+ * Failures the device sees: a router pipeline wait that runs out sets the
+ * timeout bit of an error word built into the library beside the array (one
+ * per device, shared by every call on that device). While that bit is set,
+ * calls write no weights and no indices (the partial sums may be stale);
+ * moe_gate_noalloc_check_error reads and clears it. */
 MOE_API moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x,
                                     const void* w_router, const float* bias, float* weights,
                                     int32_t* idx, void* stream);
+
+/* Read and clear the built-in error word of moe_gate_noalloc on the device
+ * that holds `x` (any device pointer of that device): synchronises `stream`,
+ * returns MOE_ERR_TIMEOUT if a call's router pipeline wait ran out since the
+ * last read, else MOE_OK (or MOE_ERR_CUDA / MOE_ERR_INVALID_ARG). Allocates
+ * no device memory. The pages have no counterpart. */
+MOE_API moe_status moe_gate_noalloc_check_error(const void* x, void* stream);
 
 /* Per-kernel timing of moe_forward, for measurement (off by default).
  * moe_stage_timing_begin(max_calls) creates max_calls * 9 CUDA events (no
@@ -197,7 +323,8 @@ MOE_API moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void
  * moe_forward_launch_count() kernels. moe_stage_timing_end(ms, n) disarms,
  * waits for the recorded events and writes to ms[i] the total milliseconds
  * kernel i (launch order: router logits, router select, dispatch rank,
- * dispatch scan, dispatch scatter, experts up, experts down, combine) took
+ * dispatch scan, dispatch positions, experts up -- with the per-expert map
+ * kernel before it, when there is one --, experts down, combine) took
  * over the recorded calls, for i < n <= 8; it returns the number of calls
  * recorded, or a negative moe_status. Single-threaded use only. */
 MOE_API moe_status moe_stage_timing_begin(int32_t max_calls);
@@ -227,15 +354,20 @@ enum {
 };
 MOE_API moe_status moe_select_expert_kernel(int32_t which);
 
-/* Test hook for the failure path of the tensor-core pipeline, process-wide,
- * off by default; the pages have no counterpart. While enabled (1), the
- * up-projection of every bf16 layer on the one-CTA tensor-core kernel has
- * its first CTA wait, before it issues anything, on a barrier phase that
- * nothing completes. The wait runs out after its 1 s limit; the launch then
- * takes the abort path every timed-out wait takes (drain the copies in
- * flight, free TMEM, return) and sets the timeout bit, so the next
- * moe_check_error() returns MOE_ERR_TIMEOUT. The rows of that CTA's tiles are
- * not written. 0 disables it; other values return MOE_ERR_INVALID_ARG. */
+/* Test hook for the failure path of the tensor-core pipelines, process-wide,
+ * off by default; the pages have no counterpart. While enabled, one kernel
+ * has its first CTA wait, before it issues anything, on a barrier phase that
+ * nothing completes:
+ *   1  the up-projection of every bf16 layer on the one-CTA tensor-core
+ *      kernel (the rows of that CTA's tiles are not written);
+ *   2  the tensor-core router logits of every bf16 layer (that CTA's partial
+ *      sums are not written).
+ * The wait runs out after its 1 s limit; the launch then takes the abort
+ * path every timed-out wait takes (drain the copies in flight, free TMEM,
+ * return) and sets the timeout bit of the call's error word, so the next
+ * moe_check_error() (moe_gate_noalloc_check_error() for moe_gate_noalloc)
+ * returns MOE_ERR_TIMEOUT. 0 disables it; other values return
+ * MOE_ERR_INVALID_ARG. */
 MOE_API moe_status moe_debug_stall_pipeline(int32_t enable);
 
 #ifdef __cplusplus

@@ -168,6 +168,9 @@ struct SelectArgs {
   float route_scale;
   float* weights;
   int32_t* idx;
+  // when set: write nothing while its timeout bit is set (the logits may be
+  // partial)
+  const uint32_t* hold_on_timeout;
 };
 
 // Values per lane VPL = ceil(E / 32); expert e lives in lane e % 32, slot e / 32.
@@ -175,6 +178,7 @@ template <int VPL>
 __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
   extern __shared__ float z_s[];  // [8][E] logits of this CTA's tokens
   __shared__ float gsc_s[8][64];
+  if (a.hold_on_timeout && (*a.hold_on_timeout & ERRBIT_TIMEOUT)) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int E = a.E;
   const int64_t t0 = (int64_t)blockIdx.x * 8;
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) 
 cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
                           const float* bias, float* weights, int32_t* idx, float* part,
                           int splits, bool simt, int num_sms, uint32_t* err_word,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool hold_on_timeout) {
   const int E = c.n_routed, D = c.dim;
   cudaError_t err;
   if (c.dtype == MOE_DT_BF16 && !simt) {
@@ -390,6 +394,7 @@ cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const v
   a.route_scale = c.route_scale;
   a.weights = weights;
   a.idx = idx;
+  a.hold_on_timeout = hold_on_timeout ? err_word : nullptr;
   unsigned blocks = (unsigned)ceil_div<int64_t>(T, 8);
   int vpl = ceil_div(E, 32);
   const size_t zs = (size_t)8 * E * sizeof(float);
@@ -407,25 +412,30 @@ cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const v
 //
 // moe_gate_noalloc runs the router with its split-k partial sums in this
 // file-scope device array instead of a caller workspace, for callers that
-// cannot allocate device memory. Every GPU that loads the library holds it
-// (4 MiB) until the process exits. Host code must not pass `g_gate_scratch`
-// itself to a kernel: on the host that name is only a stand-in; the device
-// address comes from cudaGetSymbolAddress, taken once per device.
+// cannot allocate device memory, and keeps its sticky error word (the timeout
+// bit of a router pipeline wait that ran out) in a file-scope word beside it.
+// Every GPU that loads the library holds both (4 MiB) until the process
+// exits. Host code must not pass `g_gate_scratch` or `g_gate_err` itself to a
+// kernel: on the host those names are only stand-ins; the device addresses
+// come from cudaGetSymbolAddress, taken once per device.
 
 namespace {
 constexpr size_t kGateScratchFloats = size_t(1) << 20;
 static __device__ __align__(256) float g_gate_scratch[kGateScratchFloats];
+static __device__ __align__(16) uint32_t g_gate_err;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_gate_scratch_mu;
 float* g_gate_scratch_addr[kMaxDevices] = {};
+uint32_t* g_gate_err_addr[kMaxDevices] = {};
 }  // namespace
 
 size_t gate_scratch_floats() { return kGateScratchFloats; }
 
-// Device address of the built-in scratch on the current device; looked up on
-// the first call for each device (with that device current) and cached.
-cudaError_t gate_scratch_current_device(float** out) {
+// Device addresses of the built-in scratch and of its error word on the
+// current device; looked up on the first call for each device (with that
+// device current) and cached.
+cudaError_t gate_scratch_current_device(float** scratch, uint32_t** err) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -433,11 +443,16 @@ cudaError_t gate_scratch_current_device(float** out) {
   std::lock_guard<std::mutex> lock(g_gate_scratch_mu);
   if (!g_gate_scratch_addr[dev]) {
     float* ptr = nullptr;
+    uint32_t* eptr = nullptr;
     e = cudaGetSymbolAddress((void**)&ptr, g_gate_scratch);
     if (e != cudaSuccess) return e;
+    e = cudaGetSymbolAddress((void**)&eptr, g_gate_err);
+    if (e != cudaSuccess) return e;
+    g_gate_err_addr[dev] = eptr;
     g_gate_scratch_addr[dev] = ptr;
   }
-  *out = g_gate_scratch_addr[dev];
+  *scratch = g_gate_scratch_addr[dev];
+  *err = g_gate_err_addr[dev];
   return cudaSuccess;
 }
 

@@ -7,7 +7,9 @@
 // accumulator (4 MMAs, 64 products per sum), and the epilogue warps add every
 // k-block's sums with Kahan's compensated summation in fp32 (sum plus a
 // running correction): its error stays within a few ulps of the sum however
-// many chunks are added, without fp64 work, at 4 additions per value.
+// many chunks are added, without fp64 work, at 4 additions per value (done
+// two values at a time with the packed f32x2 adds of sm_100, each lane
+// rounded exactly as a scalar add would be).
 // The tensor core therefore never sums more than 64 products, and the result
 // carries one fp32 rounding per split.
 //
@@ -35,6 +37,29 @@ constexpr uint32_t RTMEM = RNBUF * RN; // 512 columns
 constexpr size_t RSMEM = 1024 + (size_t)RSTAGES * RSTAGE + 256;
 constexpr uint32_t RIDESC = idesc_bf16(RM, RN);
 
+// Two fp32 lanes in one 64-bit register, for the packed (f32x2) adds of the
+// compensated summation: each lane is rounded to nearest like a scalar add.
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+  return v;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
 struct RouterTcArgs {
   CUtensorMap tmx;   // x [T, D]
   CUtensorMap tmw;   // W_r [E, D]
@@ -43,6 +68,10 @@ struct RouterTcArgs {
   int E;
   int kb_total;
   int kb_per_split;
+  // Test hook (moe_debug_stall_pipeline): the first CTA's MMA thread first
+  // waits on a barrier phase that nothing completes, so that wait runs out
+  // (1 s) and the launch takes its abort path.
+  int stall;
   uint32_t* err;
 };
 
@@ -107,7 +136,10 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      for (int i = 0; i < nkb; ++i) {
+      // test hook: the drain barrier is committed only after the loop
+      const bool first = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+      const bool ok = !(g.stall && first && !mbar_wait(drain, 0, abort_flag, g.err));
+      for (int i = 0; ok && i < nkb; ++i) {
         const int b = i % RNBUF;
         const uint32_t use = (uint32_t)(i / RNBUF);
         if (!mbar_wait(&tempty[b], (use & 1) ^ 1, abort_flag, g.err)) break;
@@ -130,9 +162,10 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   } else {
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    float hi[RN], lo[RN];
+    // Kahan sums of the 64 expert columns, two columns per packed register
+    uint64_t hi[RN / 2], lo[RN / 2];
 #pragma unroll
-    for (int j = 0; j < RN; ++j) hi[j] = lo[j] = 0.f;
+    for (int j = 0; j < RN / 2; ++j) hi[j] = lo[j] = 0ull;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
       const int b = i % RNBUF;
@@ -152,10 +185,10 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       tc_fence_before();
       mbar_arrive(&tempty[b]);
 #pragma unroll
-      for (int j = 0; j < RN; ++j) {  // Kahan: hi = running sum, lo = -(lost low part)
-        const float y = __fsub_rn(__uint_as_float(r[j]), lo[j]);
-        const float t = __fadd_rn(hi[j], y);
-        lo[j] = __fsub_rn(__fsub_rn(t, hi[j]), y);
+      for (int j = 0; j < RN / 2; ++j) {  // Kahan: hi = running sum, lo = -(lost low part)
+        const uint64_t y = sub2(pack2(r[2 * j], r[2 * j + 1]), lo[j]);
+        const uint64_t t = add2(hi[j], y);
+        lo[j] = sub2(sub2(t, hi[j]), y);
         hi[j] = t;
       }
     }
@@ -165,14 +198,17 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       const int nvalid = min(RN, g.E - n0);
       if (nvalid == RN && (g.E & 3) == 0) {
 #pragma unroll
-        for (int j = 0; j < RN; j += 4)
-          *reinterpret_cast<float4*>(out + j) =
-              make_float4(__fsub_rn(hi[j], lo[j]), __fsub_rn(hi[j + 1], lo[j + 1]),
-                          __fsub_rn(hi[j + 2], lo[j + 2]), __fsub_rn(hi[j + 3], lo[j + 3]));
+        for (int j = 0; j < RN / 2; j += 2) {
+          const float2 a = unpack2(sub2(hi[j], lo[j])), b = unpack2(sub2(hi[j + 1], lo[j + 1]));
+          *reinterpret_cast<float4*>(out + 2 * j) = make_float4(a.x, a.y, b.x, b.y);
+        }
       } else {
 #pragma unroll
-        for (int j = 0; j < RN; ++j)
-          if (j < nvalid) out[j] = __fsub_rn(hi[j], lo[j]);
+        for (int j = 0; j < RN / 2; ++j) {
+          const float2 a = unpack2(sub2(hi[j], lo[j]));
+          if (2 * j < nvalid) out[2 * j] = a.x;
+          if (2 * j + 1 < nvalid) out[2 * j + 1] = a.y;
+        }
       }
     }
   }
@@ -216,6 +252,7 @@ cudaError_t launch_router_logits_tc(const moe_config& c, int64_t T, const void* 
   g.E = c.n_routed;
   g.kb_total = ceil_div(c.dim, RK);
   g.kb_per_split = ceil_div(g.kb_total, splits);
+  g.stall = pipeline_stall() == STALL_ROUTER ? 1 : 0;
   g.err = err;
   const int used = ceil_div(g.kb_total, g.kb_per_split);  // every split gets >= 1 k-block
   *splits_used = used;

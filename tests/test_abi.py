@@ -110,20 +110,21 @@ def test_workspace_size_grows_with_tokens(M):
         assert b > a > 0
     cfg = inputs.CONFIGS["v3_prefill"]
     ws = M.moe_workspace_size(cfg, cfg.T)
-    # x_perm + y_perm + h dominate: 2 * T*k*D*2 + T*k*I*2 bytes
-    approx = 2 * cfg.T * 8 * 7168 * 2 + cfg.T * 8 * 2048 * 2
+    # y_perm + h dominate (no permuted copy of x): T*k*D*2 + T*k*I*2 bytes
+    approx = cfg.T * 8 * 7168 * 2 + cfg.T * 8 * 2048 * 2
     assert approx < ws < approx * 1.2
 
 
 def test_stall_hook_validates_its_argument(M):
-    assert M.raw_status("moe_debug_stall_pipeline", 2) == -1
+    assert M.raw_status("moe_debug_stall_pipeline", 3) == -1
+    assert M.raw_status("moe_debug_stall_pipeline", -1) == -1
     assert M.raw_status("moe_debug_stall_pipeline", 0) == 0
 
 
 def test_launch_count(M):
-    # bf16 on the one-CTA tensor-core kernel: each expert GEMM follows a
-    # kernel that writes its per-expert A maps
-    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 10
+    # bf16 on the one-CTA tensor-core kernel: the expert GEMMs follow one
+    # kernel that writes their per-expert A maps
+    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 9
     assert M.moe_forward_launch_count(inputs.CONFIGS["tiny_fp32"], 64) == 8
     M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_TCGEN05_PAIR)
     try:
