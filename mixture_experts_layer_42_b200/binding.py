@@ -30,16 +30,19 @@ MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX = 0, 1
 MOE_EXPERT_KERNEL_AUTO, MOE_EXPERT_KERNEL_SIMT, MOE_EXPERT_KERNEL_TCGEN05 = 0, 1, 2
 MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
+MOE_STALL_NONE, MOE_STALL_EXPERTS_UP, MOE_STALL_ROUTER = 0, 1, 2
 
 # Every symbol include/moe.h declares.
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch",
            "moe_experts_grouped", "moe_combine", "moe_forward", "moe_check_error",
            "moe_status_string", "moe_forward_launch_count", "moe_select_expert_kernel",
            "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc",
-           "moe_stage_timing_begin_every", "moe_debug_stall_pipeline")
+           "moe_stage_timing_begin_every", "moe_debug_stall_pipeline",
+           "moe_gate_noalloc_check_error", "moe_experts_grouped_gather", "moe_forward_ep",
+           "moe_cast_output", "moe_quantize_fp8", "moe_workspace_size_fp8", "moe_forward_fp8")
 
 # Kernels of moe_forward, in launch order.
-STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_scatter",
+STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_pos",
           "experts_up", "experts_down", "combine")
 
 
@@ -49,6 +52,12 @@ class moe_config(ctypes.Structure):
                 ("moe_inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32),
                 ("score", ctypes.c_int32), ("route_scale", ctypes.c_float),
                 ("has_bias", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class moe_fp8_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w1", "w3", "w2", "w1_scale", "w3_scale", "w2_scale",
+                 "ws1", "ws3", "ws2", "ws1_scale", "ws3_scale", "ws2_scale")]
 
 
 class MoEError(RuntimeError):
@@ -81,6 +90,13 @@ def _load() -> ctypes.CDLL:
         "moe_debug_stall_pipeline": [I32],
         "moe_stage_timing_end": [ctypes.POINTER(ctypes.c_float), I32],
         "moe_gate_noalloc": [C, I64, P, P, P, P, P, P],
+        "moe_gate_noalloc_check_error": [P, P],
+        "moe_experts_grouped_gather": [C, I64, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P],
+        "moe_forward_ep": [C, I64, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P],
+        "moe_cast_output": [C, I64, P, P, P],
+        "moe_quantize_fp8": [C, P, I64, I64, I32, P, P, P],
+        "moe_workspace_size_fp8": [C, I64, ctypes.POINTER(SZ)],
+        "moe_forward_fp8": [C, I64, P, P, P, ctypes.POINTER(moe_fp8_weights), P, P, P, P, SZ, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -159,8 +175,15 @@ def moe_gate_noalloc(cfg, x, w_router, bias, weights, idx, stream=None) -> None:
                                  _p(idx), _s(stream)), "moe_gate_noalloc")
 
 
+def moe_gate_noalloc_check_error(x, stream=None) -> int:
+    """Synchronise, read and clear moe_gate_noalloc's built-in error word on
+    x's device; returns the status."""
+    return int(_lib.moe_gate_noalloc_check_error(_p(x), _s(stream)))
+
+
 def moe_dispatch(cfg, idx, x, counts, offsets, src, pos, x_perm, ws, stream=None) -> None:
-    _check(_lib.moe_dispatch(_c(cfg), x.shape[0], _p(idx), _p(x), _p(counts), _p(offsets), _p(src),
+    """x_perm may be None (x is then not read; only the indices are written)."""
+    _check(_lib.moe_dispatch(_c(cfg), idx.shape[0], _p(idx), _p(x), _p(counts), _p(offsets), _p(src),
                              _p(pos), _p(x_perm), _p(ws), ws.numel(), _s(stream)), "moe_dispatch")
 
 
@@ -169,6 +192,13 @@ def moe_experts_grouped(cfg, T, x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, y
     _check(_lib.moe_experts_grouped(_c(cfg), int(T), _p(x_perm), _p(offsets), _p(w1), _p(w3), _p(w2),
                                     _p(x), _p(ws1), _p(ws3), _p(ws2), _p(y_perm), _p(s), _p(ws),
                                     ws.numel(), _s(stream)), "moe_experts_grouped")
+
+
+def moe_experts_grouped_gather(cfg, x, src, offsets, w1, w3, w2, ws1, ws3, ws2, y_perm, s, ws,
+                               stream=None) -> None:
+    _check(_lib.moe_experts_grouped_gather(_c(cfg), x.shape[0], _p(x), _p(src), _p(offsets), _p(w1),
+                                           _p(w3), _p(w2), _p(ws1), _p(ws3), _p(ws2), _p(y_perm), _p(s),
+                                           _p(ws), ws.numel(), _s(stream)), "moe_experts_grouped_gather")
 
 
 def moe_combine(cfg, y_perm, pos, weights, s, y, ws, stream=None) -> None:
@@ -181,6 +211,53 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, y, ws, weight
     _check(_lib.moe_forward(_c(cfg), x.shape[0], _p(x), _p(w_router), _p(bias), _p(w1), _p(w3),
                             _p(w2), _p(ws1), _p(ws3), _p(ws2), _p(y), _p(weights_out), _p(idx_out),
                             _p(ws), ws.numel(), _s(stream)), "moe_forward")
+
+
+def moe_forward_ep(cfg, expert_begin, expert_end, shared_local, x, w_router, bias, w1, w3, w2,
+                   ws1, ws3, ws2, y_partial, ws, weights_out=None, idx_out=None, stream=None) -> None:
+    _check(_lib.moe_forward_ep(_c(cfg), x.shape[0], int(expert_begin), int(expert_end),
+                               int(shared_local), _p(x), _p(w_router), _p(bias), _p(w1), _p(w3),
+                               _p(w2), _p(ws1), _p(ws3), _p(ws2), _p(y_partial), _p(weights_out),
+                               _p(idx_out), _p(ws), ws.numel(), _s(stream)), "moe_forward_ep")
+
+
+def moe_cast_output(cfg, y_sum, y, stream=None) -> None:
+    _check(_lib.moe_cast_output(_c(cfg), y.shape[0], _p(y_sum), _p(y), _s(stream)), "moe_cast_output")
+
+
+def moe_quantize_fp8(cfg, a, block_rows, q, scales, stream=None) -> None:
+    """a [rows, cols] (act dtype) -> q [rows, cols] e4m3 (uint8) and scales
+    [ceil(rows / block_rows), cols / 128] fp32."""
+    a2 = a.reshape(-1, a.shape[-1])
+    _check(_lib.moe_quantize_fp8(_c(cfg), _p(a2), a2.shape[0], a2.shape[1], int(block_rows), _p(q),
+                                 _p(scales), _s(stream)), "moe_quantize_fp8")
+
+
+def moe_workspace_size_fp8(cfg, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.moe_workspace_size_fp8(_c(cfg), int(T), ctypes.byref(n)), "moe_workspace_size_fp8")
+    return n.value
+
+
+def alloc_workspace_fp8(cfg, T: int, device="cuda") -> torch.Tensor:
+    ws = torch.empty(moe_workspace_size_fp8(cfg, T), dtype=torch.uint8, device=device)
+    moe_workspace_init(ws)
+    return ws
+
+
+def fp8_weights(w1, w3, w2, s1, s3, s2, ws1=None, ws3=None, ws2=None, ss1=None, ss3=None,
+                ss2=None) -> moe_fp8_weights:
+    """The C struct of FP8 expert weights from device tensors (kept alive by
+    the caller)."""
+    return moe_fp8_weights(*[None if t is None else _p(t) for t in
+                             (w1, w3, w2, s1, s3, s2, ws1, ws3, ws2, ss1, ss3, ss2)])
+
+
+def moe_forward_fp8(cfg, x, w_router, bias, fw: moe_fp8_weights, y, ws, weights_out=None,
+                    idx_out=None, stream=None) -> None:
+    _check(_lib.moe_forward_fp8(_c(cfg), x.shape[0], _p(x), _p(w_router), _p(bias), ctypes.byref(fw),
+                                _p(y), _p(weights_out), _p(idx_out), _p(ws), ws.numel(), _s(stream)),
+           "moe_forward_fp8")
 
 
 def moe_check_error(ws, stream=None) -> int:

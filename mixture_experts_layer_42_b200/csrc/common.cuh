@@ -42,8 +42,8 @@ struct WsLayout {
   size_t offsets;       // [E + 1] int32
   size_t src;           // [T * k] int32
   size_t pos;           // [T * k] int32
-  size_t x_perm;        // [T * k, D] act
-  size_t y_perm;        // [T * k, D] act
+  size_t y_perm;        // [T * k, D] act; moe_forward on the CTA-pair kernel
+                        // first holds the expert-contiguous copy of x here
   size_t s;             // [T, D] act
   size_t h;             // [T * k, I] act
   size_t hs;            // [T, I_s] act
@@ -55,6 +55,17 @@ struct WsLayout {
 };
 
 inline int act_bytes(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
+
+// Scale block edge of the FP8 expert weights and activations.
+constexpr int kFp8Block = 128;
+
+// Extra workspace regions of moe_forward_fp8, after the common layout.
+struct Fp8Layout {
+  size_t xq, xs;        // quantized x [T, D] e4m3, its scales [T, D/128] fp32
+  size_t hq, hs;        // quantized h [T*k, I], scales [T*k, I/128]
+  size_t hsq, hss;      // the shared MLP's h [T, I_s], scales [T, I_s/128]
+  size_t total;
+};
 
 // CTAs the router GEMM aims for (two per SM of a 148-SM B200).
 constexpr int kRouterTargetCtas = 296;
@@ -71,6 +82,27 @@ inline int router_splits(const moe_config& c, int64_t T) {
   if (want > maxs) want = maxs;
   if (want < 1) want = 1;
   return (int)want;
+}
+
+inline WsLayout ws_layout(const moe_config& c, int64_t T);
+
+inline Fp8Layout fp8_layout(const moe_config& c, int64_t T, size_t base) {
+  Fp8Layout L{};
+  const int64_t k = c.topk, D = c.dim, I = c.moe_inter, Is = c.shared_inter;
+  size_t off = base;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + (bytes ? bytes : 1), kWsAlign);
+    return o;
+  };
+  L.xq = take((size_t)T * D);
+  L.xs = take((size_t)T * (D / kFp8Block) * 4);
+  L.hq = take((size_t)T * k * I);
+  L.hs = take((size_t)T * k * (I / kFp8Block) * 4);
+  L.hsq = take((size_t)T * (Is > 0 ? Is : 1));
+  L.hss = take((size_t)T * (Is > 0 ? Is / kFp8Block : 1) * 4);
+  L.total = off;
+  return L;
 }
 
 inline WsLayout ws_layout(const moe_config& c, int64_t T) {
@@ -95,7 +127,6 @@ inline WsLayout ws_layout(const moe_config& c, int64_t T) {
   L.offsets = take((size_t)(E + 1) * 4);
   L.src = take((size_t)T * k * 4);
   L.pos = take((size_t)T * k * 4);
-  L.x_perm = take((size_t)T * k * D * ab);
   L.y_perm = take((size_t)T * k * D * ab);
   L.s = take((size_t)T * D * ab);
   L.h = take((size_t)T * k * I * ab);
@@ -159,7 +190,10 @@ template <> struct Vec16<float> {
 
 // Operands of one grouped expert launch ([0] routed experts, [1] shared MLP).
 struct GroupedArgs {
-  const void* a[2];     // A rows: [0] x_perm / h, [1] x / hs
+  const void* a[2];     // A rows: [0] x_perm / h (or x, see a_rows), [1] x / hs
+  // UP only: when set, row p of the routed A is row a_rows[p] of a[0] (x
+  // gathered by the dispatch's src), instead of row p of an expert-contiguous copy
+  const int32_t* a_rows;
   const void* b1[2];    // w1 / w2 stacked [E, N, K]; shared ws1 / ws2 [N_s, K_s]
   const void* b3[2];    // w3 / ws3 (UP only)
   void* out[2];         // [0] h / y_perm, [1] hs / s
@@ -177,35 +211,81 @@ void stage_mark(cudaStream_t st);
 
 // Router: logits (tensor cores for bf16 unless `simt`, else CUDA cores) into
 // `part` with at most `splits` k splits, then selection into weights / idx.
+// With `hold_on_timeout`, the selection writes nothing while the timeout bit
+// of `err` is set (moe_gate_noalloc: its partial sums may then be stale).
 cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const void* w_router,
                           const float* bias, float* weights, int32_t* idx, float* part,
-                          int splits, bool simt, int num_sms, uint32_t* err, cudaStream_t st);
+                          int splits, bool simt, int num_sms, uint32_t* err, cudaStream_t st,
+                          bool hold_on_timeout = false);
 int router_tc_splits(const moe_config& c, int64_t T, int max_splits, int num_sms);
 cudaError_t launch_router_logits_tc(const moe_config& c, int64_t T, const void* x,
                                     const void* w_router, float* part, int splits, uint32_t* err,
                                     cudaStream_t st, int* splits_used);
-// Built-in router scratch (moe_gate_noalloc): its size in floats, and its
-// device address on the current device.
+// Built-in router scratch (moe_gate_noalloc): its size in floats, and the
+// device addresses of the scratch and of its error word on the current device.
 size_t gate_scratch_floats();
-cudaError_t gate_scratch_current_device(float** out);
+cudaError_t gate_scratch_current_device(float** scratch, uint32_t** err);
 
+// x_perm may be null: then only counts, offsets, src and pos are written.
 cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
                             int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                             void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,
                             uint32_t* err, cudaStream_t st);
 cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, const int32_t* pos,
                            const float* weights, const void* s, void* y, cudaStream_t st);
+// Expert parallelism: one rank's fp32 share of y (pairs routed to its
+// n_local experts, whose offsets start at offsets_local, plus its slice of
+// the shared MLP in s), and the final cast of the summed shares.
+cudaError_t launch_combine_partial(const moe_config& c, int64_t T, const void* y_perm,
+                                   const int32_t* pos, const float* weights, const void* s,
+                                   const int32_t* offsets_local, int n_local, float* y32,
+                                   cudaStream_t st);
+cudaError_t launch_cast(const moe_config& c, int64_t T, const float* y32, void* y, cudaStream_t st);
+
+// FP8 expert weights (moe_forward_fp8): e4m3 values and the fp32 scales of
+// their 128 x 128 blocks.
+struct Fp8Weights {
+  const uint8_t *w1, *w3, *w2, *ws1, *ws3, *ws2;
+  const float *s1, *s3, *s2, *ss1, *ss3, *ss2;
+};
+// Activation rows [R, K] (act) to e4m3 with one scale per 1 x 128 block.
+cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
+                              float* scale, cudaStream_t st);
+// A matrix [R, C] (bf16 or fp32) to e4m3 with one scale per 128 x 128 block.
+cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
+                                float* scale, cudaStream_t st);
+// The FP8 expert GEMMs (gemm_fp8.cu): UP from the quantized x (routed rows
+// through src) into the quantized h, DOWN from it into y_perm and s (act).
+cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights& w,
+                               const uint8_t* xq, const float* xs, const int32_t* src,
+                               const int32_t* offsets, uint8_t* hq, float* hsc, uint8_t* hsq,
+                               float* hss, void* y_perm, void* s, uint32_t* err, int num_sms,
+                               cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
 // Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).
 enum { TC_ROWS = 0, TC_PAIR = 1 };
-// Test hook: the one-CTA up-projection's CTA 0 lets its first pipeline wait
-// run out (moe_debug_stall_pipeline).
-void set_pipeline_stall(bool on);
+// Test hook (moe_debug_stall_pipeline): which kernel's first CTA lets its
+// first pipeline wait run out -- STALL_EXPERTS_UP the one-CTA up-projection,
+// STALL_ROUTER the tensor-core router logits.
+enum { STALL_NONE = 0, STALL_EXPERTS_UP = 1, STALL_ROUTER = 2 };
+void set_pipeline_stall(int which);
+int pipeline_stall();
+// UP with src set (one-CTA kernel): the routed A rows are gathered from the
+// token rows gx [gT, k0] through src (a0 unused). row_maps: the per-expert A
+// maps written by launch_row_maps (null: none); tile_ctr: UP's tile counter.
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
-                              void* out1, const int32_t* offsets, void* row_maps, int* tile_ctr,
+                              void* out1, const int32_t* offsets, const void* gx,
+                              const int32_t* src, int64_t gT, const void* row_maps, int* tile_ctr,
                               uint32_t* err, int num_sms, cudaStream_t st);
+// Before the one-CTA expert GEMMs: per-expert copies of the down-projection's
+// A map over h [Tk, I] (at maps + E) and, when a_up is given, of the
+// up-projection's over a_up [Tk, D] (at maps), each with its row extent cut
+// at the expert's end; zeroes the up-projection's tile counter.
+cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, int D,
+                            const int32_t* offsets, int E, void* maps, int* up_tile_ctr,
+                            cudaStream_t st);
 
 }  // namespace moe

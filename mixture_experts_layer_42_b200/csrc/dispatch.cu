@@ -10,9 +10,14 @@
 //   dispatch_scan_kernel    one CTA: per-expert exclusive scan over chunks,
 //                           counts, and the exclusive scan over experts
 //                           (offsets).
-//   dispatch_scatter_kernel grid over (row slices, tokens): final positions,
-//                           src, and the copy of x[t] into its k permuted rows
-//                           with 16-byte loads and stores (x is read once).
+//   dispatch_pos_kernel     grid over the T*k pairs: final positions (pos)
+//                           and the token of every permuted row (src). The
+//                           layer's expert GEMMs read x through src, so no
+//                           permuted copy of x is made.
+//   dispatch_scatter_kernel (only when a permuted copy is asked for) grid over
+//                           (row slices, tokens): pos, src, and the copy of
+//                           x[t] into its k permuted rows with 16-byte loads
+//                           and stores (x is read once).
 #include "common.cuh"
 
 namespace moe {
@@ -141,6 +146,20 @@ dispatch_scan_kernel(int32_t* __restrict__ chunk_hist, int n_chunks, int E,
     for (int c = 0; c < n_chunks; ++c) chunk_hist[(int64_t)c * E + e] += excl;
 }
 
+__global__ void __launch_bounds__(256)
+dispatch_pos_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ pos_local,
+                    const int32_t* __restrict__ chunk_base, int64_t Tk, int k, int E,
+                    int32_t* __restrict__ pos, int32_t* __restrict__ src) {
+  const int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (q >= Tk) return;
+  const int64_t t = q / k;
+  const int pl = pos_local[q];
+  int p = -1;
+  if (pl >= 0) p = chunk_base[(t / kDispatchChunkTokens) * E + idx[q]] + pl;
+  pos[q] = p;
+  if (p >= 0) src[p] = (int32_t)t;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ pos_local,
@@ -189,6 +208,13 @@ cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, 
   dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_hist, n_chunks, E, counts, offsets);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage_mark(st);
+  if (x_perm == nullptr) {
+    const int64_t Tk = T * k;
+    dispatch_pos_kernel<<<(unsigned)ceil_div<int64_t>(Tk, 256), 256, 0, st>>>(
+        idx, pos_local, chunk_hist, Tk, k, E, pos, src);
+    stage_mark(st);
+    return cudaGetLastError();
+  }
   const int ab = act_bytes(c);
   const int nvec = D * ab / 16;
   dim3 grid((unsigned)T, (unsigned)ceil_div(nvec, 256));

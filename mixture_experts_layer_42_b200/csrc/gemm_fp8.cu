@@ -1,0 +1,633 @@
+// Grouped SwiGLU expert GEMMs with FP8 (e4m3) block-scaled weights and
+// activations, on the 5th-generation tensor cores (tcgen05.mma kind::f8f6f4).
+//
+// The pages say only that the block's other linears are FP8 ("Expert
+// scores", dtype note). The layout here is this library's: e4m3 values, one
+// power-of-two fp32 scale per 128 x 128 block of a weight matrix [out, in]
+// and per 1 x 128 block of a row of activations (the smallest scale that
+// keeps the block within 448). x is quantized once per step (quant_rows
+// kernel); h = silu(w1 x) * (w3 x) is quantized by the up-projection's
+// epilogue; each expert's output is bf16, as on the bf16 path.
+//
+// Tiles put the weights on the MMA's M side (128 rows: one scale block) and
+// up to NT tokens of one expert on its N side (rounded up to 16), so a decode
+// batch (a few tokens per expert) does little MMA work while it streams the
+// active experts' weights at half the bytes of bf16. Each 128-deep k-block
+// (one scale block) is accumulated by the tensor core into a fresh fp32 TMEM
+// buffer, and the four epilogue warps add it into register sums with the
+// product of its weight scale and each token's activation scale:
+//   sum[f, t] += s_w(e, f/128, kb) * s_x(t, kb) * sum_{k in kb} q_w[f, k] q_x[t, k]
+// (a lane of TMEM is a weight row f, a column a token t).
+//
+// One CTA per SM, 192 threads: warp 0 TMA (weights by tile, token rows by
+// tile::gather4 from the routed rows' tokens or the rows themselves; rows
+// past a tile's tokens read zeros), warp 1 MMA, warps 2-5 epilogue. Waits are
+// bounded as in the bf16 kernel (1 s, then the abort path).
+#include "tc_common.cuh"
+
+#include <cuda_fp8.h>
+
+namespace moe {
+
+namespace {
+
+using namespace tc;
+
+constexpr int QB = 128;                        // scale block edge; K per stage; weight rows per tile
+constexpr int NT = 64;                         // tokens per tile at most (MMA N)
+constexpr int FSTAGES = 4;
+constexpr int A_BYTES = NT * QB;               // 8 KB of token rows
+constexpr int W_BYTES = QB * QB;               // 16 KB per weight tile
+constexpr int FSTAGE = A_BYTES + 2 * W_BYTES;  // UP: w1 and w3 tiles; DOWN uses one
+constexpr int NTHREADS = 192;
+constexpr uint32_t FTMEM = 512;
+constexpr int MAXE = 1024;
+constexpr int MAX_KB = 64;                     // k-blocks per tile (K <= 8192)
+constexpr int NBUF_UP = 4;                     // TMEM buffers of 2 x NT columns
+constexpr int NBUF_DOWN = 8;                   // TMEM buffers of NT columns
+constexpr size_t FSMEM = 1024 + (size_t)FSTAGES * FSTAGE + 512 + 2 * (MAXE + 1) * 4 +
+                         (size_t)NT * MAX_KB * 4 + 4 * NT * 4;
+
+// kind::f8f6f4 instruction descriptor: fp32 accumulator, e4m3 A and B, both
+// K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+struct Fp8Args {
+  // token rows (uint8 [rows, K], box 128 x 1, for tile::gather4): [0] routed
+  // (UP: the quantized x, read by token through src; DOWN: the quantized h
+  // in expert order), [1] the shared MLP's (UP: quantized x; DOWN: its h)
+  CUtensorMap tmA[2];
+  CUtensorMap tmW1[2];   // weights [E, N, K] uint8, box 128 x 128 x 1: w1 (UP) / w2 (DOWN); shared E = 1
+  CUtensorMap tmW3[2];   // w3 / ws3 (UP)
+  const float* ws1[2];   // weight scales [E, N/128, K/128] of tmW1
+  const float* ws3[2];   // of tmW3
+  const float* asc[2];   // token rows' scales [rows, K/128]
+  const int32_t* src;    // routed UP: the token of each expert-order row
+  int a_rows[2];         // rows of the A tensors (an out-of-range row reads zeros)
+  void* out[2];          // UP: quantized h [rows, N] uint8; DOWN: bf16 [rows, N]
+  float* out_scale[2];   // UP: h's scales [rows, N/128]
+  int n_out[2];
+  int kdim[2];
+  const int32_t* offsets;
+  int E;
+  int t_shared;
+  uint32_t* err;
+};
+
+struct Tile {
+  int kind, e, row0, rows, n0;
+};
+
+struct Sched {
+  const int32_t* P;
+  const int32_t* off;
+  int E, nb0, nb1, ch_sh, routed, total, t_shared;
+};
+
+__device__ __forceinline__ Tile decode(const Sched& S, int i) {
+  Tile t;
+  if (i < S.routed) {
+    const int q = i / S.nb0;
+    int lo = 0, hi = S.E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (S.P[mid] <= q) lo = mid; else hi = mid;
+    }
+    const int e = lo;
+    const int mt = S.P[e + 1] - S.P[e];
+    const int l = i - S.nb0 * S.P[e];
+    const int nb = l / mt, c = l % mt;
+    t.kind = 0;
+    t.e = e;
+    t.row0 = S.off[e] + c * NT;
+    t.rows = min(NT, S.off[e + 1] - t.row0);
+    t.n0 = nb * QB;
+  } else {
+    const int l = i - S.routed;
+    const int nb = l / S.ch_sh, c = l % S.ch_sh;
+    t.kind = 1;
+    t.e = 0;
+    t.row0 = c * NT;
+    t.rows = min(NT, S.t_shared - t.row0);
+    t.n0 = nb * QB;
+  }
+  return t;
+}
+
+__device__ __forceinline__ int round16(int r) { return (r + 15) & ~15; }
+
+// Smallest s with amax <= 448 * 2^s (0 for amax == 0): amax = m 2^e with
+// 0.5 <= m < 1, so s = e - 9, plus one when 2m > 1.75.
+__device__ __forceinline__ int block_exp(float amax) {
+  if (!(amax > 0.f)) return 0;
+  int e;
+  const float m = frexpf(amax, &e);
+  return e - 9 + (2.f * m > 1.75f ? 1 : 0);
+}
+
+// (Values are brought into range with ldexpf(v, -s): the reciprocal 2^-s of
+// a tiny block's scale would overflow fp32, the scaled value does not.)
+__device__ __forceinline__ uint8_t to_e4m3(float v) {
+  return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
+
+// Named barrier 1 over the four epilogue warps that also ORs a flag across
+// them, so that every warp takes the same abort decision before the next
+// barrier (a warp that left alone would leave the others waiting).
+__device__ __forceinline__ bool epi_sync_any(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag)
+      : "memory");
+  return r != 0;
+}
+
+template <bool UP>
+__global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  constexpr int NBUF = UP ? NBUF_UP : NBUF_DOWN;
+  constexpr int BUF_COLS = UP ? 2 * NT : NT;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + FSTAGES * FSTAGE);
+  uint64_t* empty = full + FSTAGES;
+  uint64_t* tfull = empty + FSTAGES;
+  uint64_t* tempty = tfull + NBUF;
+  uint64_t* drain = tempty + NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* P = reinterpret_cast<int32_t*>(tiles + FSTAGES * FSTAGE + 512);
+  int32_t* off = P + MAXE + 1;
+  float* tsc = reinterpret_cast<float*>(off + MAXE + 1);  // [NT][MAX_KB] token scales of the tile
+  float* red = tsc + NT * MAX_KB;                         // [4][NT] per-warp maxima
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int E = g.E;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < FSTAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+      for (int b = 0; b < NBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+      mbar_init(drain, 1);
+      *abort_flag = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    // token chunks per expert and their exclusive prefix
+    const int per = (E + 31) / 32;
+    int lsum = 0;
+    for (int u = 0; u < per; ++u) {
+      const int e = lane * per + u;
+      if (e < E) {
+        const int o0 = g.offsets[e], o1 = g.offsets[e + 1];
+        off[e] = o0;
+        if (e == E - 1) off[E] = o1;
+        lsum += (o1 - o0 + NT - 1) / NT;
+      }
+    }
+    int incl = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int p = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += p;
+    }
+    int run = incl - lsum;
+    for (int u = 0; u < per; ++u) {
+      const int e = lane * per + u;
+      if (e < E) {
+        P[e] = run;
+        run += (g.offsets[e + 1] - g.offsets[e] + NT - 1) / NT;
+      }
+    }
+    if (lane == 31) P[E] = incl;
+    __syncwarp();
+  } else if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(FTMEM));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  Sched S;
+  S.P = P;
+  S.off = off;
+  S.E = E;
+  S.nb0 = g.n_out[0] / QB;
+  S.nb1 = g.t_shared > 0 ? g.n_out[1] / QB : 0;
+  S.ch_sh = (g.t_shared + NT - 1) / NT;
+  S.t_shared = g.t_shared;
+  S.routed = S.nb0 * P[E];
+  S.total = S.routed + S.nb1 * S.ch_sh;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    // lane 0: barriers and the weight tiles; lanes 0..n16/4-1: 4 token rows
+    // each by tile::gather4
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int i = blockIdx.x; i < S.total; i += gridDim.x) {
+      const Tile t = decode(S, i);
+      const int kb_n = g.kdim[t.kind] / QB;
+      const int n16 = round16(t.rows);
+      const int n_g = n16 / 4;
+      const uint32_t tx = (uint32_t)(n16 * QB + (UP ? 2 : 1) * W_BYTES);
+      int r[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = 4 * lane + q;
+        const int row = t.row0 + j;
+        int a = g.a_rows[t.kind];                        // out of range: zeros
+        if (j < t.rows) a = (UP && t.kind == 0 && g.src != nullptr) ? g.src[row] : row;
+        r[q] = a;
+      }
+      for (int kb = 0; kb < kb_n; ++kb) {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        uint8_t* sa = tiles + s * FSTAGE;
+        uint8_t* sw = sa + A_BYTES;
+        if (lane == 0) {
+          mbar_expect_tx(&full[s], tx);
+          tma_load_3d(sw, &g.tmW1[t.kind], &full[s], kb * QB, t.n0, t.e);
+          if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], kb * QB, t.n0, t.e);
+        }
+        __syncwarp();
+        if (lane < n_g)
+          tma_gather4(sa + lane * (4 * QB), &g.tmA[t.kind], &full[s], kb * QB, r[0], r[1], r[2], r[3]);
+        ++issued;
+        if (++s == FSTAGES) { s = 0; ph ^= 1; }
+      }
+      if (!ok) break;
+    }
+    if (!ok && lane == 0) {
+      for (int j = 0; j < FSTAGES; ++j) {
+        const int n = issued / FSTAGES + (j < issued % FSTAGES ? 1 : 0);
+        if (n > 0) mbar_drain(&full[j], (uint32_t)((n - 1) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0, u = 0;  // u: k-blocks issued so far (TMEM buffer rotation)
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < S.total; i += gridDim.x) {
+        const Tile t = decode(S, i);
+        const int kb_n = g.kdim[t.kind] / QB;
+        const uint32_t idesc = idesc_e4m3(QB, round16(t.rows));
+        for (int kb = 0; kb < kb_n; ++kb, ++u) {
+          const int b = u % NBUF;
+          const uint32_t use = (uint32_t)(u / NBUF);
+          if (!mbar_wait(&tempty[b], (use & 1) ^ 1, abort_flag, g.err)) { ok = false; break; }
+          tc_fence_after();
+          if (!mbar_wait(&full[s], ph, abort_flag, g.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(tiles + s * FSTAGE);
+          const uint32_t w0 = a0 + A_BYTES;
+          const uint32_t d = tmem_base + (uint32_t)(b * BUF_COLS);
+#pragma unroll
+          for (int kk = 0; kk < QB / 32; ++kk) {
+            mma_f8(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, kk != 0 ? 1u : 0u);
+            if (UP) mma_f8(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc,
+                           kk != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+          tc_commit(&tfull[b]);
+          if (++s == FSTAGES) { s = 0; ph ^= 1; }
+        }
+      }
+      tc_commit(drain);
+      mbar_drain(drain, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int f = quad * 32 + lane;      // this thread's weight row (TMEM lane) in the tile
+    const int et = threadIdx.x - 64;     // 0..127 among the epilogue threads
+    int u = 0;
+    for (int i = blockIdx.x; i < S.total; i += gridDim.x) {
+      const Tile t = decode(S, i);
+      const int kb_n = g.kdim[t.kind] / QB;
+      const int n16 = round16(t.rows);
+      bool ok = true;
+      // the tile's token scales for every k-block, into shared memory
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int q = et; q < NT * kb_n; q += 128) {
+        const int j = q / kb_n, kb = q % kb_n;
+        float v = 0.f;
+        if (j < t.rows) {
+          const int row = t.row0 + j;
+          const int a = (UP && t.kind == 0 && g.src != nullptr) ? g.src[row] : row;
+          v = g.asc[t.kind][(int64_t)a * kb_n + kb];
+        }
+        tsc[j * MAX_KB + kb] = v;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int nbw = g.n_out[t.kind] / QB;
+      const float* sw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
+      const float* sw3 = UP ? g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n : nullptr;
+      float sa[NT], sb[UP ? NT : 1];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) { sa[j] = 0.f; if (UP) sb[j] = 0.f; }
+      for (int kb = 0; kb < kb_n; ++kb, ++u) {
+        const int b = u % NBUF;
+        const uint32_t use = (uint32_t)(u / NBUF);
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&tfull[b], use & 1, abort_flag, g.err) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * BUF_COLS);
+        const float c1 = __ldg(sw1 + kb);
+        const float c3 = UP ? __ldg(sw3 + kb) : 0.f;
+#pragma unroll
+        for (int j0 = 0; j0 < NT; j0 += 16) {
+          if (j0 < n16) {
+            uint32_t ra[16], rb[16];
+            tmem_ld16(tb + j0, ra);
+            if (UP) tmem_ld16(tb + NT + j0, rb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float xs = tsc[(j0 + q) * MAX_KB + kb];
+              sa[j0 + q] = fmaf(__uint_as_float(ra[q]), c1 * xs, sa[j0 + q]);
+              if (UP) sb[j0 + q] = fmaf(__uint_as_float(rb[q]), c3 * xs, sb[j0 + q]);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[b]);
+      }
+      // one decision for all four warps: stop if any of them gave up
+      if (epi_sync_any(!ok)) break;
+      if (UP) {
+        // h = silu(a) * b, quantized per token over this tile's 128 features
+        // (one 1 x 128 block of h's row)
+        uint8_t* hq = reinterpret_cast<uint8_t*>(g.out[t.kind]);
+        float* hs = g.out_scale[t.kind];
+        const int nbh = g.n_out[t.kind] / QB;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (j >= n16) break;
+          const float h = silu_f(sa[j]) * sb[j];
+          sa[j] = h;
+          float m = fabsf(h);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) red[quad * NT + j] = m;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {   // unrolled: sa stays in registers
+          if (j < t.rows) {
+            const float amax = fmaxf(fmaxf(red[j], red[NT + j]), fmaxf(red[2 * NT + j], red[3 * NT + j]));
+            const int se = block_exp(amax);
+            const int64_t row = t.row0 + j;
+            hq[row * g.n_out[t.kind] + t.n0 + f] = to_e4m3(ldexpf(sa[j], -se));
+            if (et == 0) hs[row * nbh + t.n0 / QB] = ldexpf(1.f, se);
+          }
+        }
+      } else {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          if (j < t.rows)
+            out[(int64_t)(t.row0 + j) * g.n_out[t.kind] + t.n0 + f] = __float2bfloat16_rn(sa[j]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(FTMEM));
+  }
+}
+
+// Rows [R, K] (act) to e4m3 with one power-of-two scale per 1 x 128 block:
+// one warp per block, 4 elements per lane.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int64_t R, int K,
+                                                         uint8_t* __restrict__ q,
+                                                         float* __restrict__ scale) {
+  const int kbn = K / QB;
+  const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (blk >= R * kbn) return;
+  const int64_t r = blk / kbn;
+  const int kb = (int)(blk % kbn);
+  const T* p = a + r * K + kb * QB + lane * 4;
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = to_f32(p[i]);
+  float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const int se = block_exp(m);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(ldexpf(v[i], -se)) << (8 * i);
+  reinterpret_cast<uint32_t*>(q + r * K + kb * QB)[lane] = packed;
+  if (lane == 0) scale[r * kbn + kb] = ldexpf(1.f, se);
+}
+
+// A bf16 / fp32 matrix [R, C] to e4m3 with one power-of-two scale per
+// 128 x 128 block (the weights' layout): one CTA per block, 256 threads.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_blocks_kernel(const T* __restrict__ a, int64_t R, int C,
+                                                           uint8_t* __restrict__ q,
+                                                           float* __restrict__ scale) {
+  __shared__ float wmax[8];
+  const int64_t br = blockIdx.y;
+  const int bc = blockIdx.x;
+  const int nbc = C / QB;
+  const int64_t r0 = br * QB;
+  const int rows = (int)(R - r0 < QB ? R - r0 : QB);
+  float m = 0.f;
+  for (int i = threadIdx.x; i < rows * QB; i += 256) {
+    const int rr = i / QB, cc = i % QB;
+    m = fmaxf(m, fabsf(to_f32(a[(r0 + rr) * C + bc * QB + cc])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (threadIdx.x % 32 == 0) wmax[threadIdx.x / 32] = m;
+  __syncthreads();
+  m = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+  const int se = block_exp(m);
+  for (int i = threadIdx.x; i < rows * QB; i += 256) {
+    const int rr = i / QB, cc = i % QB;
+    const int64_t o = (r0 + rr) * C + bc * QB + cc;
+    q[o] = to_e4m3(ldexpf(to_f32(a[o]), -se));  // exact: a power-of-two step, no overflow
+  }
+  if (threadIdx.x == 0) scale[br * nbc + bc] = ldexpf(1.f, se);
+}
+
+bool map_u8_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K};
+  cuuint32_t box[2] = {QB, 1};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {K, N, E};
+  cuuint64_t strides[2] = {K, N * K};
+  cuuint32_t box[3] = {QB, QB, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
+                              float* scale, cudaStream_t st) {
+  const int64_t warps = R * (K / QB);
+  if (warps == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)ceil_div<int64_t>(warps * 32, 256);
+  if (c.dtype == MOE_DT_BF16)
+    quant_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)a, R, K, q, scale);
+  else
+    quant_rows_kernel<float><<<blocks, 256, 0, st>>>((const float*)a, R, K, q, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
+                                float* scale, cudaStream_t st) {
+  dim3 grid((unsigned)(C / QB), (unsigned)ceil_div<int64_t>(R, QB));
+  if (bf16)
+    quant_blocks_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)a, R, C, q, scale);
+  else
+    quant_blocks_kernel<float><<<grid, 256, 0, st>>>((const float*)a, R, C, q, scale);
+  return cudaGetLastError();
+}
+
+// The FP8 expert GEMMs of one layer: UP reads the quantized x (routed rows
+// by token through src, shared rows directly) and writes the quantized h and
+// hs; DOWN reads them and writes y_perm and s (bf16).
+cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights& w,
+                               const uint8_t* xq, const float* xs, const int32_t* src,
+                               const int32_t* offsets, uint8_t* hq, float* hsc, uint8_t* hsq,
+                               float* hss, void* y_perm, void* s, uint32_t* err, int num_sms,
+                               cudaStream_t st) {
+  const int E = c.n_routed, D = c.dim, I = c.moe_inter, Is = c.shared_inter;
+  const int64_t Tk = T * c.topk;
+  const bool sh = Is > 0;
+  cudaError_t e;
+  for (int pass = 0; pass < 2; ++pass) {
+    const bool up = pass == 0;
+    Fp8Args g;
+    memset(&g, 0, sizeof(g));
+    const int n0 = up ? I : D, k0 = up ? D : I, n1 = up ? Is : D, k1 = up ? D : Is;
+    if (up) {
+      if (!map_u8_rows(&g.tmA[0], xq, (uint64_t)T, (uint64_t)D)) return cudaErrorInvalidValue;
+      g.a_rows[0] = (int)T;
+      g.asc[0] = xs;
+      g.src = src;
+      if (!map_u8_weights(&g.tmW1[0], w.w1, E, I, D)) return cudaErrorInvalidValue;
+      if (!map_u8_weights(&g.tmW3[0], w.w3, E, I, D)) return cudaErrorInvalidValue;
+      g.ws1[0] = w.s1;
+      g.ws3[0] = w.s3;
+      g.out[0] = hq;
+      g.out_scale[0] = hsc;
+      if (sh) {
+        g.tmA[1] = g.tmA[0];
+        g.a_rows[1] = (int)T;
+        g.asc[1] = xs;
+        if (!map_u8_weights(&g.tmW1[1], w.ws1, 1, Is, D)) return cudaErrorInvalidValue;
+        if (!map_u8_weights(&g.tmW3[1], w.ws3, 1, Is, D)) return cudaErrorInvalidValue;
+        g.ws1[1] = w.ss1;
+        g.ws3[1] = w.ss3;
+        g.out[1] = hsq;
+        g.out_scale[1] = hss;
+      }
+    } else {
+      if (!map_u8_rows(&g.tmA[0], hq, (uint64_t)Tk, (uint64_t)I)) return cudaErrorInvalidValue;
+      g.a_rows[0] = (int)Tk;
+      g.asc[0] = hsc;
+      if (!map_u8_weights(&g.tmW1[0], w.w2, E, D, I)) return cudaErrorInvalidValue;
+      g.ws1[0] = w.s2;
+      g.out[0] = y_perm;
+      if (sh) {
+        if (!map_u8_rows(&g.tmA[1], hsq, (uint64_t)T, (uint64_t)Is)) return cudaErrorInvalidValue;
+        g.a_rows[1] = (int)T;
+        g.asc[1] = hss;
+        if (!map_u8_weights(&g.tmW1[1], w.ws2, 1, D, Is)) return cudaErrorInvalidValue;
+        g.ws1[1] = w.ss2;
+        g.out[1] = s;
+      }
+    }
+    if (!sh) {  // no shared group: its maps are never used, keep them valid
+      g.tmA[1] = g.tmA[0];
+      g.tmW1[1] = g.tmW1[0];
+      g.tmW3[1] = g.tmW3[0];
+    }
+    if (!up) {  // DOWN reads one weight tile per stage
+      g.tmW3[0] = g.tmW1[0];
+      g.tmW3[1] = g.tmW1[1];
+    }
+    g.n_out[0] = n0;
+    g.n_out[1] = sh ? n1 : n0;
+    g.kdim[0] = k0;
+    g.kdim[1] = sh ? k1 : k0;
+    g.offsets = offsets;
+    g.E = E;
+    g.t_shared = sh ? (int)T : 0;
+    g.err = err;
+    const int64_t bound = (int64_t)(n0 / QB) * ((Tk + NT - 1) / NT + E) +
+                          (sh ? (int64_t)(n1 / QB) * ((T + NT - 1) / NT) : 0);
+    const int grid = (int)(bound < num_sms ? bound : num_sms);
+    if (grid > 0) {
+      if (up) {
+        e = cudaFuncSetAttribute(grouped_fp8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)FSMEM);
+        if (e != cudaSuccess) return e;
+        grouped_fp8_kernel<true><<<grid, NTHREADS, FSMEM, st>>>(g);
+      } else {
+        e = cudaFuncSetAttribute(grouped_fp8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)FSMEM);
+        if (e != cudaSuccess) return e;
+        grouped_fp8_kernel<false><<<grid, NTHREADS, FSMEM, st>>>(g);
+      }
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    stage_mark(st);
+  }
+  return cudaSuccess;
+}
+
+}  // namespace moe

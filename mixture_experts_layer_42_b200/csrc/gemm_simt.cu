@@ -4,8 +4,10 @@
 // MLP; SwiGLU body E(x) = w2 (silu(w1 x) * (w3 x))) as two grouped launches:
 //   UP:   h[r, n] = silu(sum_k A[r,k] w1[e,n,k]) * (sum_k A[r,k] w3[e,n,k])
 //   DOWN: out[r, n] = sum_k h[r,k] w2[e,n,k]
-// Group e owns rows [offsets[e], offsets[e+1]) of A; a last group, the shared
-// expert, owns all T rows of its own A. Tiles of 64 rows x 64 columns; each
+// Group e owns rows [offsets[e], offsets[e+1]) of A (for UP, either an
+// expert-contiguous copy of the token rows or the token rows themselves read
+// through the dispatch's src); a last group, the shared expert, owns all T
+// rows of its own A. Tiles of 64 rows x 64 columns; each
 // CTA finds its group from the device offsets (no host round trip).
 //
 // This path serves the fp32 layer (tensor cores have no full-precision fp32
@@ -84,6 +86,9 @@ __global__ void __launch_bounds__(256) grouped_simt_kernel(const GroupedArgs g) 
   const int n0 = blockIdx.y * SBN;
   if (n0 >= N) return;
   const T* A = (const T*)g.a[kind];
+  // row of A that holds row r of this group (gathered rows for routed UP)
+  const int32_t* a_rows = (UP && kind == 0) ? g.a_rows : nullptr;
+  auto arow = [&](int64_t r) -> int64_t { return a_rows ? (int64_t)a_rows[r] : r; };
   const T* B1 = (const T*)g.b1[kind] + (int64_t)e * N * K;
   const T* B3 = UP ? (const T*)g.b3[kind] + (int64_t)e * N * K : nullptr;
   T* out = (T*)g.out[kind];
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(256) grouped_simt_kernel(const GroupedArgs g) 
       const int i = tid + 256 * r;
       const int rr = i / SBK, kk = i % SBK;
       const int k = k0 + kk;
-      As[kk][rr] = (rr < rows && k < K) ? to_f32(A[(row0 + rr) * K + k]) : 0.f;
+      As[kk][rr] = (rr < rows && k < K) ? to_f32(A[arow(row0 + rr) * K + k]) : 0.f;
       const int n = n0 + rr;
       B1s[kk][rr] = (n < N && k < K) ? to_f32(B1[(int64_t)n * K + k]) : 0.f;
       if (UP) B3s[kk][rr] = (n < N && k < K) ? to_f32(B3[(int64_t)n * K + k]) : 0.f;

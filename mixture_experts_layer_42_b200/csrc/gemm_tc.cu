@@ -132,7 +132,7 @@ struct TileQueue {
 // measured slower at prefill.
 constexpr int SWAP_ROWS = 64;
 __device__ __forceinline__ bool swap_tail(const Tile& t, const TcArgs& g) {
-  return t.kind == 0 && t.only && t.rows <= SWAP_ROWS && g.row_maps != nullptr;
+  return t.kind == 0 && t.only && t.rows <= SWAP_ROWS && (g.row_maps != nullptr || g.src != nullptr);
 }
 __device__ __forceinline__ int tail_n(int rows) { return (rows + 15) & ~15; }
 
@@ -222,46 +222,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      int s = 0, issued = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      TileQueue Q;
-      const bool dyn = g.tile_ctr != nullptr;
-      // the next tile is claimed a few k-blocks before the current one ends,
-      // so the atomic's round trip overlaps the current tile's loads
-      int next = dyn ? atomicAdd(g.tile_ctr, 1) : (int)blockIdx.x;
-      for (;;) {
-        const int i = next;
-        if (dyn) {
-          // hand the tile's index to the MMA and epilogue warps
-          if (!mbar_wait(&qempty[Q.q], Q.ph ^ 1, abort_flag, g.err)) { ok = false; break; }
-          tq[Q.q] = i;
-          mbar_arrive(&qfull[Q.q]);
-          Q.advance();
-        } else {
-          next = i + (int)gridDim.x;
+    // Lane 0 claims tiles, waits for free stages and loads B (and A, when A
+    // is loaded by tile). When the routed A rows are gathered from the token
+    // rows, every lane brings 4 of the tile's rows per stage (tile::gather4):
+    // lane l rows 4l..4l+3.
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    TileQueue Q;
+    const bool dyn = g.tile_ctr != nullptr;
+    // the next tile is claimed a few k-blocks before the current one ends,
+    // so the atomic's round trip overlaps the current tile's loads
+    int next = 0;
+    if (lane == 0) next = dyn ? atomicAdd(g.tile_ctr, 1) : (int)blockIdx.x;
+    next = __shfl_sync(0xffffffffu, next, 0);
+    for (;;) {
+      const int i = next;
+      if (dyn) {
+        // hand the tile's index to the MMA and epilogue warps
+        int w = 1;
+        if (lane == 0) {
+          w = mbar_wait(&qempty[Q.q], Q.ph ^ 1, abort_flag, g.err) ? 1 : 0;
+          if (w) {
+            tq[Q.q] = i;
+            mbar_arrive(&qfull[Q.q]);
+          }
         }
-        if (i >= S.total) break;
-        const Tile t = decode(S, i);
-        const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
-        const int kb_claim = kb_n > 4 ? kb_n - 4 : 0;
-        // an expert's last, partial tile reads zeros past its rows, not the
-        // next expert's; a swapped tile's box is only tail_n(rows) rows high
-        const CUtensorMap* ta = &g.tmA[t.kind];
-        uint32_t tx = STAGE_BYTES;
-        if (t.kind == 0 && t.rows < BM && g.row_maps != nullptr) {
-          ta = g.row_maps + t.e;
-          tmap_acquire(ta);
-          if (swap_tail(t, g)) tx = (uint32_t)(tail_n(t.rows) * BK * 2 + B_TILE);
-        }
-        for (int kb = 0; kb < kb_n; ++kb) {
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        Q.advance();
+      } else {
+        next = i + (int)gridDim.x;
+      }
+      if (i >= S.total) break;
+      const Tile t = decode(S, i);
+      const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
+      const int kb_claim = kb_n > 4 ? kb_n - 4 : 0;
+      const bool swap = swap_tail(t, g);
+      // an expert's last, partial tile reads zeros past its rows, not the
+      // next expert's; a swapped tile's box is only tail_n(rows) rows high
+      const CUtensorMap* ta = &g.tmA[t.kind];
+      uint32_t tx = STAGE_BYTES;
+      if (swap) tx = (uint32_t)(tail_n(t.rows) * BK * 2 + B_TILE);
+      const bool gath = UP && t.kind == 0 && g.src != nullptr;
+      int gr0 = 0, gr1 = 0, gr2 = 0, gr3 = 0, n_g = 0;
+      if (gath) {
+        // this lane's four rows: their tokens, or the out-of-range row gT
+        // (zeros) past the expert's end
+        n_g = (swap ? tail_n(t.rows) : BM) / 4;
+        const int r = 4 * lane;
+        gr0 = r + 0 < t.rows ? g.src[t.row0 + r + 0] : g.gT;
+        gr1 = r + 1 < t.rows ? g.src[t.row0 + r + 1] : g.gT;
+        gr2 = r + 2 < t.rows ? g.src[t.row0 + r + 2] : g.gT;
+        gr3 = r + 3 < t.rows ? g.src[t.row0 + r + 3] : g.gT;
+      } else if (t.kind == 0 && t.rows < BM && g.row_maps != nullptr) {
+        ta = g.row_maps + t.e;
+        if (lane == 0) tmap_acquire(ta);
+      }
+      for (int kb = 0; kb < kb_n; ++kb) {
+        int w = 1;
+        if (lane == 0) {
           if (dyn && kb == kb_claim) next = atomicAdd(g.tile_ctr, 1);
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err)) { ok = false; break; }
-          uint8_t* sa = tiles + s * STAGE_BYTES;
-          uint8_t* sb = sa + A_TILE;
+          w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        uint8_t* sa = tiles + s * STAGE_BYTES;
+        uint8_t* sb = sa + A_TILE;
+        if (lane == 0) {
           mbar_expect_tx(&full[s], tx);
-          tma_load_2d(sa, ta, &full[s], kb * BK, t.row0);
+          if (!gath) tma_load_2d(sa, ta, &full[s], kb * BK, t.row0);
           if (UP && g.b13[t.kind]) {
             tma_load_4d(sb, &g.tmB13[t.kind], &full[s], kb * BK, t.n0, t.e, 0);
           } else if (UP) {
@@ -270,17 +298,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
           } else {
             tma_load_3d(sb, &g.tmB1[t.kind], &full[s], kb * BK, t.n0, t.e);
           }
-          ++issued;
-          if (++s == STAGES) { s = 0; ph ^= 1; }
         }
-        if (!ok) break;
+        __syncwarp();
+        if (gath && lane < n_g)
+          tma_gather4(sa + lane * (4 * BK * 2), &g.tmG, &full[s], kb * BK, gr0, gr1, gr2, gr3);
+        ++issued;
+        if (++s == STAGES) { s = 0; ph ^= 1; }
       }
-      if (!ok) {
-        // let every copy still in flight land before the CTA exits
-        for (int j = 0; j < STAGES; ++j) {
-          const int n = issued / STAGES + (j < issued % STAGES ? 1 : 0);
-          if (n > 0) mbar_drain(&full[j], (uint32_t)((n - 1) & 1));
-        }
+      if (!ok) break;
+      if (dyn) next = __shfl_sync(0xffffffffu, next, 0);
+    }
+    if (!ok && lane == 0) {
+      // let every copy still in flight land before the CTA exits
+      for (int j = 0; j < STAGES; ++j) {
+        const int n = issued / STAGES + (j < issued % STAGES ? 1 : 0);
+        if (n > 0) mbar_drain(&full[j], (uint32_t)((n - 1) & 1));
       }
     }
   } else if (warp == 1) {
@@ -480,19 +512,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   }
 }
 
-// Per-expert copies of the routed A map with the row extent cut at the
-// expert's end: one warp per expert edits a copy in shared memory and
-// publishes it to global memory with a release fence for the tensor-map proxy.
-__global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ CUtensorMap base,
+// Per-expert copies of an A map with the row extent cut at the expert's end:
+// one warp per expert edits a copy in shared memory and publishes it to
+// global memory with a release fence for the tensor-map proxy. blockIdx.y
+// selects the map: 0 the down-projection's (rows of h), 1 the
+// up-projection's (rows of the expert-contiguous copy of x; not launched when
+// the up-projection gathers its rows from x).
+struct RowMapArgs {
+  CUtensorMap base[2];
+  CUtensorMap* maps[2];
+};
+
+__global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ RowMapArgs a,
                                                              const int32_t* __restrict__ offsets,
-                                                             int E, CUtensorMap* maps,
-                                                             int* tile_ctr) {
+                                                             int E, int* tile_ctr) {
   __shared__ __align__(128) CUtensorMap sm[8];
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *tile_ctr = 0;  // the GEMM's tile queue restarts
+  const int which = blockIdx.y;
+  if (blockIdx.x == 0 && which == 0 && threadIdx.x == 0) *tile_ctr = 0;  // the up-projection's queue restarts
   const int e = blockIdx.x * 8 + w;
   if (e >= E) return;  // whole warps
-  reinterpret_cast<uint32_t*>(&sm[w])[lane] = reinterpret_cast<const uint32_t*>(&base)[lane];
+  reinterpret_cast<uint32_t*>(&sm[w])[lane] = reinterpret_cast<const uint32_t*>(&a.base[which])[lane];
   __syncwarp();
   if (lane == 0) {
     const int end = offsets[e + 1];
@@ -512,37 +552,64 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
   __syncwarp();
   asm volatile(
       "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], "
-      "[%1], 128;" ::"l"(maps + e),
+      "[%1], 128;" ::"l"(a.maps[which] + e),
       "r"(smem_u32(&sm[w]))
       : "memory");
 }
 
 }  // namespace
 
-// A: routed rows [Tk, K0] and shared rows [T, K1]; B1/B3 stacked [E, N0, K0]
-// and shared [N1, K1]; outputs [Tk, N0] and [T, N1]. `kind` picks the
-// kernel: TC_ROWS this one (128-row tiles), TC_PAIR the CTA-pair kernel
-// (256-row tiles, gemm_tc2.cu).
 // Test hook state (moe_debug_stall_pipeline).
-static bool g_stall = false;
-void set_pipeline_stall(bool on) { g_stall = on; }
+static int g_stall = STALL_NONE;
+void set_pipeline_stall(int which) { g_stall = which; }
+int pipeline_stall() { return g_stall; }
 
+cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, int D,
+                            const int32_t* offsets, int E, void* maps, int* up_tile_ctr,
+                            cudaStream_t st) {
+  RowMapArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!tc::map_2d(&a.base[0], h, (uint64_t)Tk, (uint64_t)I, BM)) return cudaErrorInvalidValue;
+  a.maps[0] = static_cast<CUtensorMap*>(maps) + E;
+  if (a_up != nullptr) {
+    if (!tc::map_2d(&a.base[1], a_up, (uint64_t)Tk, (uint64_t)D, BM)) return cudaErrorInvalidValue;
+    a.maps[1] = static_cast<CUtensorMap*>(maps);
+  }
+  dim3 grid((unsigned)((E + 7) / 8), a_up != nullptr ? 2u : 1u);
+  build_row_maps_kernel<<<grid, 256, 0, st>>>(a, offsets, E, up_tile_ctr);
+  return cudaGetLastError();
+}
+
+// A: routed rows [Tk, K0] (or, for UP, the token rows gx [gT, K0] gathered
+// through src) and shared rows [T_sh, K1]; B1/B3 stacked [E, N0, K0] and
+// shared [N1, K1]; outputs [Tk, N0] and [T_sh, N1]. `kind` picks the kernel:
+// TC_ROWS this one (128-row tiles), TC_PAIR the CTA-pair kernel (256-row
+// tiles, gemm_tc2.cu; no gathering, row maps or tile counter).
 cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E, const void* a0,
                               const void* a1, const void* b1_0, const void* b3_0, const void* b1_1,
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
-                              void* out1, const int32_t* offsets, void* row_maps, int* tile_ctr,
+                              void* out1, const int32_t* offsets, const void* gx,
+                              const int32_t* src, int64_t gT, const void* row_maps, int* tile_ctr,
                               uint32_t* err, int num_sms, cudaStream_t st) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
   const bool pair = kind == TC_PAIR;
+  const bool gather = up && !pair && src != nullptr;
+  if (!gather && a0 == nullptr) return cudaErrorInvalidValue;
   // Weight rows per TMA box: one CTA loads all 256 MMA rows of B (UP: 128 w1
   // + 128 w3); in a pair each CTA loads 128 (UP: 64 w1 + 64 w3).
   const uint32_t box_n = up ? (pair ? BN / 4 : BN / 2) : (pair ? BN / 2 : BN);
   const uint32_t box_a = BM;
   const bool has_sh = T_sh > 0;
-  if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a)) return cudaErrorInvalidValue;
-  if (pair && !tc::map_2d(&g.tmA64[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a / 2))
-    return cudaErrorInvalidValue;
+  if (gather) {
+    if (!tc::map_gather(&g.tmG, gx, (uint64_t)gT, (uint64_t)k0)) return cudaErrorInvalidValue;
+    g.src = src;
+    g.gT = (int)gT;
+  } else {
+    if (!tc::map_2d(&g.tmA[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a)) return cudaErrorInvalidValue;
+    if (pair && !tc::map_2d(&g.tmA64[0], a0, (uint64_t)Tk, (uint64_t)k0, box_a / 2))
+      return cudaErrorInvalidValue;
+  }
   if (!tc::map_3d(&g.tmB1[0], b1_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
     return cudaErrorInvalidValue;
   if (up && !tc::map_3d(&g.tmB3[0], b3_0, (uint64_t)E, (uint64_t)n0, (uint64_t)k0, box_n))
@@ -605,19 +672,16 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
     stage_mark(st);
     return cudaSuccess;
   }
-  if (row_maps != nullptr && tile_ctr != nullptr && E > 0) {
-    g.row_maps = static_cast<const CUtensorMap*>(row_maps);
+  if (E > 0) {
+    // per-expert A maps (built before the launch; not needed when gathering)
+    g.row_maps = gather ? nullptr : static_cast<const CUtensorMap*>(row_maps);
     // Tiles in order from a counter for the up-projection: its long tiles
-    // (K = D) keep the CTAs that share weight and x_perm tiles in step, where
+    // (K = D) keep the CTAs that share weight and A tiles in step, where
     // round-robin lets them drift apart and re-read from HBM (UP read 1.15x
     // its algorithmic DRAM bytes at prefill). The down-projection's tiles
     // (K = I) are short enough that the hand-off costs more than it saves.
     g.tile_ctr = up ? tile_ctr : nullptr;
-    g.stall = up && g_stall ? 1 : 0;
-    build_row_maps_kernel<<<(E + 7) / 8, 256, 0, st>>>(g.tmA[0], offsets, E,
-                                                       static_cast<CUtensorMap*>(row_maps), tile_ctr);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    g.stall = up && g_stall == STALL_EXPERTS_UP ? 1 : 0;
   }
   if (up) {
     e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -92,10 +92,13 @@ moe_status bind_device(cudaStream_t s, const void* ptr) {
   return MOE_OK;
 }
 
-moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* offsets,
-                       const void* w1, const void* w3, const void* w2, const void* x,
-                       const void* ws1, const void* ws3, const void* ws2, void* y_perm, void* s,
-                       void* h, void* hs, void* row_maps, uint32_t* err, cudaStream_t st) {
+// The expert GEMMs. The routed A rows come from x_perm (an expert-contiguous
+// copy of x) or, when x_perm is null, are gathered from x through src.
+moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* src,
+                       const int32_t* offsets, const void* w1, const void* w3, const void* w2,
+                       const void* x, const void* ws1, const void* ws3, const void* ws2,
+                       void* y_perm, void* s, void* h, void* hs, void* row_maps, uint32_t* err,
+                       cudaStream_t st) {
   const int64_t Tk = T * c.topk;
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
@@ -104,16 +107,28 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
     // the same GPU, the pairs' 256-row tiles pad enough extra rows at the
     // DeepSeek-V3 prefill shape to lose to single CTAs under the power cap.
     const int kind = g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR ? TC_PAIR : TC_ROWS;
+    if (kind == TC_PAIR && x_perm == nullptr) return MOE_ERR_UNSUPPORTED;
     // tile counters of the up and down launches, after the 2 x E row maps
     int* ctr = reinterpret_cast<int*>(static_cast<uint8_t*>(row_maps) + (size_t)2 * c.n_routed * 128);
-    cudaError_t e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
-                                      c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets,
-                                      row_maps, ctr, err, num_sms_current(), st);
+    void* maps_down = static_cast<uint8_t*>(row_maps) + (size_t)c.n_routed * 128;
+    cudaError_t e = cudaSuccess;
+    if (kind == TC_ROWS) {
+      // one small launch before both GEMMs: each expert's A maps with the row
+      // extent cut at its end (the down-projection's over h, and the
+      // up-projection's over x_perm unless it gathers from x), and the
+      // up-projection's tile counter reset
+      e = launch_row_maps(h, Tk, c.moe_inter, x_perm, c.dim, offsets, c.n_routed, row_maps, ctr, st);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
+                          c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets, x,
+                          x_perm ? nullptr : src, T, kind == TC_ROWS ? row_maps : nullptr, ctr, err,
+                          num_sms_current(), st);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
-                          c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets,
-                          static_cast<uint8_t*>(row_maps) + (size_t)c.n_routed * 128, ctr + 16,
-                          err, num_sms_current(), st);
+                          c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, nullptr,
+                          nullptr, 0, kind == TC_ROWS ? maps_down : nullptr, nullptr, err,
+                          num_sms_current(), st);
     return cuda_status(e);
   }
   GroupedArgs g;
@@ -121,7 +136,8 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
   g.offsets = offsets;
   g.E = c.n_routed;
   g.t_shared = sh ? T : 0;
-  g.a[0] = x_perm; g.a[1] = x;
+  g.a[0] = x_perm ? x_perm : x; g.a[1] = x;
+  g.a_rows = x_perm ? nullptr : src;
   g.b1[0] = w1; g.b1[1] = ws1;
   g.b3[0] = w3; g.b3[1] = ws3;
   g.out[0] = h; g.out[1] = hs;
@@ -130,6 +146,7 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
   cudaError_t e = launch_grouped_simt(c, T, true, g, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   g.a[0] = h; g.a[1] = hs;
+  g.a_rows = nullptr;
   g.b1[0] = w2; g.b1[1] = ws2;
   g.b3[0] = nullptr; g.b3[1] = nullptr;
   g.out[0] = y_perm; g.out[1] = s;
@@ -152,6 +169,39 @@ struct StageTiming {
 };
 StageTiming g_timing;
 
+// Arms the per-kernel events for one forward call when stage timing is on
+// (one call in `every`); counts the call if all its events were recorded.
+struct TimedCall {
+  explicit TimedCall(cudaStream_t s) {
+    StageTiming& T = g_timing;
+    T.in_forward = T.on && T.calls < T.max_calls && T.seen % T.every == 0;
+    if (T.on) ++T.seen;
+    if (T.in_forward) T.marks = 0;
+    stage = s;
+  }
+  void start();
+  ~TimedCall() {
+    StageTiming& T = g_timing;
+    if (T.in_forward) {
+      if (T.marks == T.per_call) ++T.calls;
+      T.in_forward = false;
+    }
+  }
+  cudaStream_t stage;
+};
+
+// Average rows per expert up to which moe_forward gathers the up-projection's
+// rows from x instead of copying them (the swapped-tile limit of the one-CTA
+// tensor-core kernel).
+constexpr int64_t kGatherRows = 64;
+
+bool fp8_shapes_ok(const moe_config& c) {
+  const int B = kFp8Block;
+  if (c.dtype != MOE_DT_BF16) return false;
+  if (c.dim % B || c.moe_inter % B || c.shared_inter % B) return false;
+  return c.dim / B <= 64 && c.moe_inter / B <= 64 && c.shared_inter / B <= 64;
+}
+
 }  // namespace
 
 void stage_mark(cudaStream_t st) {
@@ -160,6 +210,10 @@ void stage_mark(cudaStream_t st) {
   cudaEventRecord(T.ev[(size_t)T.calls * T.per_call + T.marks], st);
   ++T.marks;
 }
+
+namespace {
+void TimedCall::start() { stage_mark(stage); }
+}  // namespace
 
 }  // namespace moe
 
@@ -204,9 +258,10 @@ moe_status moe_dispatch(const moe_config* cfg, int64_t T, const int32_t* idx, co
                         void* x_perm, void* ws, size_t ws_bytes, void* stream) {
   moe_status st = check_config(cfg, T);
   if (st != MOE_OK) return st;
-  if (!aligned16(idx) || !aligned16(x) || !aligned16(counts) || !aligned16(offsets) ||
-      !aligned16(src) || !aligned16(pos) || !aligned16(x_perm))
+  if (!aligned16(idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(src) ||
+      !aligned16(pos))
     return MOE_ERR_INVALID_ARG;
+  if (x_perm && (!aligned16(x_perm) || !aligned16(x))) return MOE_ERR_INVALID_ARG;
   WsLayout L;
   if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
   if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
@@ -231,7 +286,30 @@ moe_status moe_experts_grouped(const moe_config* cfg, int64_t T, const void* x_p
   WsLayout L;
   if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
   if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
-  return run_experts(*cfg, T, x_perm, offsets, w1, w3, w2, x, ws1, ws3, ws2, y_perm, s,
+  return run_experts(*cfg, T, x_perm, nullptr, offsets, w1, w3, w2, x, ws1, ws3, ws2, y_perm, s,
+                     at<void>(ws, L.h), at<void>(ws, L.hs), at<void>(ws, L.row_maps),
+                     at<uint32_t>(ws, L.header), (cudaStream_t)stream);
+}
+
+moe_status moe_experts_grouped_gather(const moe_config* cfg, int64_t T, const void* x,
+                                      const int32_t* src, const int32_t* offsets, const void* w1,
+                                      const void* w3, const void* w2, const void* ws1,
+                                      const void* ws3, const void* ws2, void* y_perm, void* s,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(src) || !aligned16(offsets) || !aligned16(w1) ||
+      !aligned16(w3) || !aligned16(w2) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->shared_inter > 0 && (!aligned16(ws1) || !aligned16(ws3) || !aligned16(ws2) ||
+                                !aligned16(s)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->dtype == MOE_DT_BF16 && g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR)
+    return MOE_ERR_UNSUPPORTED;
+  WsLayout L;
+  if ((st = check_ws(*cfg, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = bind_device((cudaStream_t)stream, ws)) != MOE_OK) return st;
+  return run_experts(*cfg, T, nullptr, src, offsets, w1, w3, w2, x, ws1, ws3, ws2, y_perm, s,
                      at<void>(ws, L.h), at<void>(ws, L.hs), at<void>(ws, L.row_maps),
                      at<uint32_t>(ws, L.header), (cudaStream_t)stream);
 }
@@ -270,22 +348,8 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   if ((st = check_ws(c, T, ws, ws_bytes, &L)) != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   if ((st = bind_device(s, ws)) != MOE_OK) return st;
-  StageTiming& TM = g_timing;
-  TM.in_forward = TM.on && TM.calls < TM.max_calls && TM.seen % TM.every == 0;
-  if (TM.on) ++TM.seen;
-  if (TM.in_forward) {
-    TM.marks = 0;
-    stage_mark(s);
-  }
-  struct EndCall {
-    StageTiming& t;
-    ~EndCall() {
-      if (t.in_forward) {
-        if (t.marks == t.per_call) ++t.calls;
-        t.in_forward = false;
-      }
-    }
-  } end_call{TM};
+  TimedCall timed(s);
+  timed.start();
   float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   uint32_t* err = at<uint32_t>(ws, L.header);
@@ -295,16 +359,184 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
     return MOE_ERR_CUDA;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   int32_t* pos = at<int32_t>(ws, L.pos);
-  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, at<int32_t>(ws, L.src),
-                      pos, at<void>(ws, L.x_perm), at<int32_t>(ws, L.chunk_hist),
-                      at<int32_t>(ws, L.pos_local), L.n_chunks, err, s) != cudaSuccess)
+  int32_t* src = at<int32_t>(ws, L.src);
+  // The routed token rows reach the up-projection either straight from x
+  // through src (tile::gather4, four rows per copy) or from an
+  // expert-contiguous copy made by the dispatch (one tile copy per stage).
+  // Measured on B200 at the DeepSeek-V3 shape: with 128-row tiles the 32
+  // gathers per stage bound the up-projection by the TMA's copy rate (10.9
+  // against 4.8 ms at T = 8192), while batches of at most kGatherRows rows per
+  // expert (decode) run their few rows as swapped tiles and gather 4 to 16 rows
+  // per stage at no cost. So batches that average more rows per expert, and
+  // the CTA-pair option, take the copy; it lives in y_perm's space, which is
+  // free until the down-projection writes it.
+  const bool big = T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed;
+  const bool copy_rows = c.dtype == MOE_DT_BF16 &&
+                         (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR || big);
+  void* x_perm = copy_rows ? at<void>(ws, L.y_perm) : nullptr;
+  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, src, pos, x_perm,
+                      at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
+                      s) != cudaSuccess)
     return MOE_ERR_CUDA;
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
-  st = run_experts(c, T, at<void>(ws, L.x_perm), offsets, w1, w3, w2, x, ws1, ws3, ws2,
+  st = run_experts(c, T, x_perm, src, offsets, w1, w3, w2, x, ws1, ws3, ws2,
                    at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
                    at<void>(ws, L.row_maps), err, s);
   if (st != MOE_OK) return st;
+  return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
+}
+
+moe_status moe_forward_ep(const moe_config* cfg, int64_t T, int32_t expert_begin,
+                          int32_t expert_end, int32_t shared_local, const void* x,
+                          const void* w_router, const float* bias, const void* w1, const void* w3,
+                          const void* w2, const void* ws1, const void* ws3, const void* ws2,
+                          float* y_partial, float* weights_out, int32_t* idx_out, void* ws,
+                          size_t ws_bytes, void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (expert_begin < 0 || expert_end <= expert_begin || expert_end > c.n_routed)
+    return MOE_ERR_INVALID_ARG;
+  const int q = c.dtype == MOE_DT_BF16 ? 8 : 4;
+  if (shared_local < 0 || shared_local > c.shared_inter || shared_local % q) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(w3) ||
+      !aligned16(w2) || !aligned16(y_partial))
+    return MOE_ERR_INVALID_ARG;
+  if (c.has_bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if (shared_local > 0 && (!aligned16(ws1) || !aligned16(ws3) || !aligned16(ws2)))
+    return MOE_ERR_INVALID_ARG;
+  if ((weights_out && !aligned16(weights_out)) || (idx_out && !aligned16(idx_out)))
+    return MOE_ERR_INVALID_ARG;
+  if (c.dtype == MOE_DT_BF16 && g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR)
+    return MOE_ERR_UNSUPPORTED;
+  WsLayout L;
+  if ((st = check_ws(c, T, ws, ws_bytes, &L)) != MOE_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = bind_device(s, ws)) != MOE_OK) return st;
+  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+  uint32_t* err = at<uint32_t>(ws, L.header);
+  // every rank routes every token over all experts (the gate is replicated)
+  if (launch_router(c, T, x, w_router, bias, weights, idx, at<float>(ws, L.router_part),
+                    L.router_splits, g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
+                    err, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* pos = at<int32_t>(ws, L.pos);
+  int32_t* src = at<int32_t>(ws, L.src);
+  // gathered rows or a permuted copy, by the same rule as moe_forward
+  const bool big = T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed;
+  void* x_perm = (c.dtype == MOE_DT_BF16 && big) ? at<void>(ws, L.y_perm) : nullptr;
+  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, src, pos, x_perm,
+                      at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
+                      s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // this rank's experts are a contiguous run of the expert order: the
+  // grouped GEMMs see them as a layer of n_local experts whose offsets start
+  // at expert_begin's, and the shared MLP as one of width shared_local
+  moe_config lc = c;
+  lc.n_routed = expert_end - expert_begin;
+  lc.shared_inter = shared_local;
+  const int32_t* off_local = offsets + expert_begin;
+  void* sbuf = shared_local > 0 ? at<void>(ws, L.s) : nullptr;
+  st = run_experts(lc, T, x_perm, src, off_local, w1, w3, w2, x, ws1, ws3, ws2,
+                   at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
+                   at<void>(ws, L.row_maps), err, s);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_combine_partial(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf,
+                                            off_local, lc.n_routed, y_partial, s));
+}
+
+moe_status moe_cast_output(const moe_config* cfg, int64_t T, const float* y_sum, void* y,
+                           void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!aligned16(y_sum) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if ((st = bind_device((cudaStream_t)stream, y)) != MOE_OK) return st;
+  return cuda_status(launch_cast(*cfg, T, y_sum, y, (cudaStream_t)stream));
+}
+
+moe_status moe_quantize_fp8(const moe_config* cfg, const void* a, int64_t rows, int64_t cols,
+                            int32_t block_rows, void* q, float* scales, void* stream) {
+  if (!cfg || (cfg->dtype != MOE_DT_BF16 && cfg->dtype != MOE_DT_F32)) return MOE_ERR_INVALID_ARG;
+  if (rows < 1 || cols < kFp8Block || cols % kFp8Block || cols > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  if (block_rows != 1 && block_rows != kFp8Block) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(q) || !aligned16(scales)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  moe_status st = bind_device(s, a);
+  if (st != MOE_OK) return st;
+  if (block_rows == 1)
+    return cuda_status(launch_quant_rows(*cfg, a, rows, (int)cols, static_cast<uint8_t*>(q), scales, s));
+  return cuda_status(launch_quant_blocks(cfg->dtype == MOE_DT_BF16, a, rows, (int)cols,
+                                         static_cast<uint8_t*>(q), scales, s));
+}
+
+moe_status moe_workspace_size_fp8(const moe_config* cfg, int64_t T, size_t* bytes) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  if (!fp8_shapes_ok(*cfg)) return MOE_ERR_UNSUPPORTED;
+  *bytes = fp8_layout(*cfg, T, ws_layout(*cfg, T).total).total;
+  return MOE_OK;
+}
+
+moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
+                           const float* bias, const moe_fp8_weights* w, void* y,
+                           float* weights_out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status st = check_config(cfg, T);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (!fp8_shapes_ok(c)) return MOE_ERR_UNSUPPORTED;
+  if (!w || !aligned16(x) || !aligned16(w_router) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->w1) || !aligned16(w->w3) || !aligned16(w->w2) || !aligned16(w->w1_scale) ||
+      !aligned16(w->w3_scale) || !aligned16(w->w2_scale))
+    return MOE_ERR_INVALID_ARG;
+  if (c.shared_inter > 0 &&
+      (!aligned16(w->ws1) || !aligned16(w->ws3) || !aligned16(w->ws2) ||
+       !aligned16(w->ws1_scale) || !aligned16(w->ws3_scale) || !aligned16(w->ws2_scale)))
+    return MOE_ERR_INVALID_ARG;
+  if (c.has_bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if ((weights_out && !aligned16(weights_out)) || (idx_out && !aligned16(idx_out)))
+    return MOE_ERR_INVALID_ARG;
+  WsLayout L = ws_layout(c, T);
+  const Fp8Layout F = fp8_layout(c, T, L.total);
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < F.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = bind_device(s, ws)) != MOE_OK) return st;
+  TimedCall timed(s);
+  timed.start();
+  float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
+  uint32_t* err = at<uint32_t>(ws, L.header);
+  if (launch_router(c, T, x, w_router, bias, weights, idx, at<float>(ws, L.router_part),
+                    L.router_splits, g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
+                    err, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* pos = at<int32_t>(ws, L.pos);
+  int32_t* src = at<int32_t>(ws, L.src);
+  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, src, pos, nullptr,
+                      at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
+                      s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // x to e4m3 once per step (its kernel is timed with the up-projection)
+  uint8_t* xq = at<uint8_t>(ws, F.xq);
+  float* xs = at<float>(ws, F.xs);
+  if (launch_quant_rows(c, x, T, c.dim, xq, xs, s) != cudaSuccess) return MOE_ERR_CUDA;
+  Fp8Weights fw{static_cast<const uint8_t*>(w->w1), static_cast<const uint8_t*>(w->w3),
+                static_cast<const uint8_t*>(w->w2), static_cast<const uint8_t*>(w->ws1),
+                static_cast<const uint8_t*>(w->ws3), static_cast<const uint8_t*>(w->ws2),
+                w->w1_scale, w->w3_scale, w->w2_scale, w->ws1_scale, w->ws3_scale, w->ws2_scale};
+  const bool sh = c.shared_inter > 0;
+  void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
+  if (launch_grouped_fp8(c, T, fw, xq, xs, src, offsets, at<uint8_t>(ws, F.hq), at<float>(ws, F.hs),
+                         at<uint8_t>(ws, F.hsq), at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf,
+                         err, num_sms_current(), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
 }
 
@@ -338,12 +570,12 @@ const char* moe_status_string(moe_status st) {
 
 int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
   if (check_config(cfg, T) != MOE_OK) return -1;
-  // router: logits + select; dispatch: rank + scan + scatter; experts: up +
-  // down, each after a kernel that writes its per-expert A maps when the
+  // router: logits + select; dispatch: rank + scan + positions; experts: up
+  // + down, after one kernel that writes the per-expert A maps when the
   // one-CTA tensor-core kernel runs; combine
   const bool row_maps = cfg->dtype == MOE_DT_BF16 && (g_expert_kernel == MOE_EXPERT_KERNEL_AUTO ||
                                                       g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05);
-  return 2 + 3 + 2 + (row_maps ? 2 : 0) + 1;
+  return 2 + 3 + 2 + (row_maps ? 1 : 0) + 1;
 }
 
 moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
@@ -358,13 +590,31 @@ moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, con
   cudaStream_t s = (cudaStream_t)stream;
   if ((st = bind_device(s, x)) != MOE_OK) return st;
   float* scratch = nullptr;
-  if (gate_scratch_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t* err = nullptr;
+  if (gate_scratch_current_device(&scratch, &err) != cudaSuccess) return MOE_ERR_CUDA;
   int splits = router_splits(*cfg, T);
   const int64_t fit = (int64_t)gate_scratch_floats() / per_split;
   if (splits > fit) splits = (int)fit;
+  // a router wait that runs out sets the timeout bit of the built-in error
+  // word; the selection then writes no routing until the word is cleared
   return cuda_status(launch_router(*cfg, T, x, w_router, bias, weights, idx, scratch, splits,
                                    g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
-                                   nullptr, s));
+                                   err, s, /*hold_on_timeout=*/true));
+}
+
+moe_status moe_gate_noalloc_check_error(const void* x, void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  moe_status st = bind_device(s, x);
+  if (st != MOE_OK) return st;
+  float* scratch = nullptr;
+  uint32_t* err = nullptr;
+  if (gate_scratch_current_device(&scratch, &err) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, err, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(err, 0, sizeof(word), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  return (word & ERRBIT_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_OK;
 }
 
 moe_status moe_stage_timing_begin(int32_t max_calls) {
@@ -407,8 +657,9 @@ int32_t moe_stage_timing_end(float* ms, int32_t n) {
 }
 
 moe_status moe_debug_stall_pipeline(int32_t enable) {
-  if (enable != 0 && enable != 1) return MOE_ERR_INVALID_ARG;
-  set_pipeline_stall(enable != 0);
+  if (enable != STALL_NONE && enable != STALL_EXPERTS_UP && enable != STALL_ROUTER)
+    return MOE_ERR_INVALID_ARG;
+  set_pipeline_stall(enable);
   return MOE_OK;
 }
 

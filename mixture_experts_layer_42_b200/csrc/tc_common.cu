@@ -28,6 +28,10 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K, uint32_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool map_gather(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K) {
+  return map_2d(m, ptr, rows, K, 1);
+}
+
 bool map_3d(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K, uint32_t box_n) {
   auto fn = encode_fn();
   if (!fn) return false;

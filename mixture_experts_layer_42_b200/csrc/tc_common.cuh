@@ -124,6 +124,21 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, ui
       : "memory");
 }
 
+// Four rows of a 2D tensor (a map whose box is 64 elements x 1 row) into
+// shared memory as one 4-row, 512-byte piece of a 128-byte-swizzled tile: row
+// coordinates r0..r3 may be anything (an out-of-range row reads zeros), the
+// column coordinate c0 selects the 64-element slice. The swizzle follows the
+// destination address, so `dst` at a 512-byte offset inside a 1024-byte-
+// aligned tile gives the same bytes as one tile load of those rows.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tm, uint64_t* bar, int c0,
+                                            int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // Make a tensor map written to global memory through the generic proxy
 // (tensormap.cp_fenceproxy ... release) visible to this thread's TMA loads.
 __device__ __forceinline__ void tmap_acquire(const void* map) {
@@ -266,15 +281,24 @@ struct TcArgs {
   // Boxes hold 128 rows of each for one CTA, 64 for a CTA pair.
   CUtensorMap tmB13[2];
   int b13[2];
+  // UP, one-CTA kernel: when `src` is set, the routed A rows are not read
+  // from an expert-contiguous copy but gathered from the token rows x [gT, K]
+  // through tmG (box 64 x 1 row, tile::gather4): row p of the expert order is
+  // token src[p]; rows past an expert's end are given the out-of-range row gT
+  // and read as zeros.
+  CUtensorMap tmG;
+  const int32_t* src;
+  int gT;
   void* out[2];
   int n_out[2];         // output columns: UP I / I_s, DOWN D / D
   int kdim[2];          // reduction depth: UP D / D, DOWN I / I_s
   const int32_t* offsets;
   // One-CTA kernel: [E] copies of tmA[0] whose row extent ends at the
   // expert's last row (offsets[e + 1]), so that a tile reaching past it reads
-  // zeros there; null when not built.
+  // zeros there (written by build_row_maps_kernel before the launch); null
+  // when the routed A rows are gathered or the maps are not built.
   const CUtensorMap* row_maps;
-  // One-CTA kernel: the launch's tile counter (zeroed by the row-map kernel
+  // One-CTA kernel: the launch's tile counter (zeroed by build_row_maps_kernel
   // before it); CTAs take tiles from it in order instead of round-robin by
   // CTA index. Null: round-robin.
   int* tile_ctr;
@@ -297,6 +321,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
 // 2D bf16 map over a row-major [rows, K] matrix, box 64 (K) x box_rows,
 // 128-byte swizzle, zero fill out of bounds.
 bool map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K, uint32_t box_rows);
+
+// 2D bf16 map over a row-major [rows, K] matrix for tile::gather4 loads: box
+// 64 (K) x 1 row, 128-byte swizzle, zero fill out of bounds.
+bool map_gather(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K);
 
 // 3D bf16 map over stacked matrices [E, N, K], box 64 (K) x box_n x 1.
 bool map_3d(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K, uint32_t box_n);

@@ -52,6 +52,8 @@ class MoEConfig:
     route_scale: float
     dtype: str             # "f32" | "bf16"
     seed: int = 0
+    fp8: bool = False      # expert weights in the FP8 block-scaled layout (quantized from
+                           # the drawn bf16 weights by the library)
 
     @property
     def shared_inter(self) -> int:
@@ -91,6 +93,11 @@ CONFIGS = {
     "v3_zipf": MoEConfig("v3_zipf", T=8192, dim=7168, n_routed=256, n_groups=8,
                          topk_groups=4, topk=8, moe_inter=2048, n_shared=1,
                          score="sigmoid", bias="zipf", route_scale=2.5, dtype="bf16"),
+    # The decode batch with its expert weights in the FP8 block-scaled layout.
+    "v3_decode_fp8": MoEConfig("v3_decode_fp8", T=128, dim=7168, n_routed=256, n_groups=8,
+                               topk_groups=4, topk=8, moe_inter=2048, n_shared=1,
+                               score="sigmoid", bias="normal", route_scale=2.5, dtype="bf16",
+                               fp8=True),
 }
 
 # Zipf exponent of the skewed workload and the scale beta of its bias. Beta was

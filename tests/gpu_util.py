@@ -77,8 +77,10 @@ class Layer:
         assert M.moe_check_error(ws) == M.MOE_OK
         return y, wts, idx
 
-    def split(self, idx, wts):
-        """dispatch + experts + combine with the given routing (device tensors)."""
+    def split(self, idx, wts, gather=False):
+        """dispatch + experts + combine with the given routing (device tensors);
+        with `gather`, the experts read x through src (moe_experts_grouped_gather)
+        instead of an expert-contiguous copy."""
         c, T = self.cfg, self.T
         dev = self.device
         ws = M.alloc_workspace(c, T, dev)
@@ -87,14 +89,18 @@ class Layer:
         offsets = torch.empty(c.n_routed + 1, dtype=torch.int32, device=dev)
         src = torch.empty(Tk, dtype=torch.int32, device=dev)
         pos = torch.empty(Tk, dtype=torch.int32, device=dev)
-        x_perm = torch.empty(Tk, c.dim, dtype=c.torch_dtype, device=dev)
+        x_perm = None if gather else torch.empty(Tk, c.dim, dtype=c.torch_dtype, device=dev)
         y_perm = torch.empty(Tk, c.dim, dtype=c.torch_dtype, device=dev)
         sh = c.shared_inter > 0
         s = torch.empty(T, c.dim, dtype=c.torch_dtype, device=dev) if sh else None
         y = torch.empty(T, c.dim, dtype=c.torch_dtype, device=dev)
         w1, w3, w2, ws1, ws3, ws2 = self.w
         M.moe_dispatch(c, idx, self.x, counts, offsets, src, pos, x_perm, ws)
-        M.moe_experts_grouped(c, T, x_perm, offsets, w1, w3, w2, self.x, ws1, ws3, ws2, y_perm, s, ws)
+        if gather:
+            M.moe_experts_grouped_gather(c, self.x, src, offsets, w1, w3, w2, ws1, ws3, ws2, y_perm, s, ws)
+        else:
+            M.moe_experts_grouped(c, T, x_perm, offsets, w1, w3, w2, self.x, ws1, ws3, ws2, y_perm, s,
+                                  ws)
         M.moe_combine(c, y_perm, pos, wts, s, y, ws)
         st = M.moe_check_error(ws)
         return y, dict(counts=counts, offsets=offsets, src=src, pos=pos, x_perm=x_perm,

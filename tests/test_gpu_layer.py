@@ -55,12 +55,10 @@ def test_fp32_forward_variants(kw):
     assert err < 1e-4
 
 
-def test_softmax_nogroup_sampled_tokens():
-    cfg = inputs.CONFIGS["softmax_nogroup"]
-    L = Layer(cfg)
-    rng = np.random.default_rng(0)
-    tokens = np.sort(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 254, replace=False)]))
-    err, r, nt = forward_parity(L, tokens=np.unique(tokens))
+def test_softmax_nogroup_all_tokens():
+    # the softmax workload at full size (T = 4096, D = 2048, 64 experts,
+    # top-6, two shared experts), every token against the oracle
+    err, r, nt = forward_parity(Layer(inputs.CONFIGS["softmax_nogroup"]))
     assert err < 2e-2
 
 
@@ -143,12 +141,14 @@ def _dispatch_check(L, idx_np, out):
     assert (out["offsets"].cpu().numpy() == d["offsets"]).all()
     assert (out["src"].cpu().numpy() == d["src"]).all()
     assert (out["pos"].cpu().numpy().reshape(idx_np.shape) == d["pos"]).all()
-    xp = out["x_perm"].cpu()
-    assert torch.equal(xp, L.x.cpu()[torch.from_numpy(d["src"])])
+    if out.get("x_perm") is not None:
+        xp = out["x_perm"].cpu()
+        assert torch.equal(xp, L.x.cpu()[torch.from_numpy(d["src"])])
 
 
+@pytest.mark.parametrize("copy_rows", [True, False], ids=["x_perm", "indices_only"])
 @pytest.mark.parametrize("name,T", [("tiny_fp32", None), ("v3_decode", None), ("v3_zipf", 2048)])
-def test_dispatch_matches_oracle(name, T):
+def test_dispatch_matches_oracle(name, T, copy_rows):
     cfg = inputs.CONFIGS[name]
     L = Layer(cfg, T=T, weights=(None,) * 6)
     r = L.oracle_route()
@@ -162,8 +162,9 @@ def test_dispatch_matches_oracle(name, T):
                offsets=torch.empty(c.n_routed + 1, dtype=torch.int32, device="cuda"),
                src=torch.empty(Tk, dtype=torch.int32, device="cuda"),
                pos=torch.empty(Tk, dtype=torch.int32, device="cuda"),
-               x_perm=torch.empty(Tk, c.dim, dtype=c.torch_dtype, device="cuda"))
-    M.moe_dispatch(c, idx, L.x, out["counts"], out["offsets"], out["src"], out["pos"], out["x_perm"], ws)
+               x_perm=torch.empty(Tk, c.dim, dtype=c.torch_dtype, device="cuda") if copy_rows else None)
+    M.moe_dispatch(c, idx, L.x if copy_rows else None, out["counts"], out["offsets"], out["src"],
+                   out["pos"], out["x_perm"], ws)
     assert M.moe_check_error(ws) == M.MOE_OK
     _dispatch_check(L, r["idx"], out)
 
@@ -283,6 +284,49 @@ def test_tensor_core_vs_simt(kw):
         assert np.median(rel) < 1e-2
 
 
+@pytest.mark.parametrize("which", [M.MOE_EXPERT_KERNEL_TCGEN05, M.MOE_EXPERT_KERNEL_SIMT],
+                         ids=["tensor_core", "cuda_core"])
+@pytest.mark.parametrize("kw", [{}, dict(T=77), dict(T=640, dim=512, moe_inter=256),
+                                dict(T=2000, n_routed=8, n_groups=2, topk_groups=1, topk=2),
+                                dict(T=200, dim=256, moe_inter=128, n_routed=1024, n_groups=32,
+                                     topk_groups=8, topk=32),
+                                dict(n_shared=0)])
+def test_gathered_rows_match_the_permuted_copy_bitwise(kw, which):
+    # the experts reading x through src (tile::gather4 on the tensor cores)
+    # see the same A rows as with the expert-contiguous copy, padding rows
+    # included (zeros both ways), so every output is bit for bit the same
+    cfg = bf16_small(**kw)
+    L, r, idx, w = _experts_case(cfg)
+    with _kernel(which):
+        y_c, out_c = L.split(idx, w)
+        y_g, out_g = L.split(idx, w, gather=True)
+    assert out_c["status"] == M.MOE_OK and out_g["status"] == M.MOE_OK
+    assert torch.equal(y_c, y_g)
+    assert torch.equal(out_c["y_perm"], out_g["y_perm"])
+    if cfg.n_shared:
+        assert torch.equal(out_c["s"], out_g["s"])
+    err = check_y(cfg, to_np(y_g), L.oracle_y(r, np.arange(L.T)))
+    assert err < 2e-2
+
+
+def test_gathered_experts_need_the_one_cta_kernel():
+    cfg = bf16_small(T=64)
+    L, r, idx, w = _experts_case(cfg)
+    with _kernel(M.MOE_EXPERT_KERNEL_TCGEN05_PAIR):
+        with pytest.raises(M.MoEError) as e:
+            L.split(idx, w, gather=True)
+    assert e.value.status == M.MOE_ERR_UNSUPPORTED
+
+
+def test_forward_on_the_cta_pair_kernel():
+    # moe_forward on the CTA-pair option dispatches an expert-contiguous copy
+    # of x into y_perm's space, which the down-projection then overwrites
+    cfg = bf16_small(T=700, dim=512, moe_inter=256)
+    with _kernel(M.MOE_EXPERT_KERNEL_TCGEN05_PAIR):
+        err, r, nt = forward_parity(Layer(cfg))
+    assert err < 2e-2
+
+
 def test_pair_and_single_cta_kernels_agree_bitwise():
     # the two tensor-core kernels add the same products in the same k order
     # into fp32 accumulators, so their bf16 outputs are identical
@@ -352,10 +396,10 @@ def test_w1_w3_memory_layouts(layout):
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32", "softmax_nogroup"])
-def test_routing_profile_driver_runs(name, capsys):
-    # the profiling driver of the non-expert kernels (no expert weights)
-    from mixture_experts_layer_42_b200 import profile_routing
-    profile_routing.main(["--config", name, "--iters", "2"])
+def test_bench_routing_only_mode_runs(name, capsys):
+    # the benchmark's mode for profiling the non-expert kernels (no expert weights)
+    import bench
+    bench.main(["--routing-only", "--config", name, "--iters", "2"])
     assert "done" in capsys.readouterr().out
 
 
