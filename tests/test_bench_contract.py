@@ -23,6 +23,14 @@ def _check_reference_line(d, n_gpus):
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["n_gpus"] == n_gpus and d["steps"] == 2 and d["warmup"] == 1
     assert d["config"]["workload"] == "tiny_fp32"
+    # the same config object the GPU arm prints for this workload
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_42_b200 import inputs
+    cfg = inputs.CONFIGS["tiny_fp32"]
+    assert d["config"] == bench.config_dict(cfg, n_gpus, "auto", bench.l2_note(cfg, cfg.n_routed))
+    # ms_per_step is the measured time of one step of the sample, not T / value
+    assert d["ms_per_step"] * 1e-3 * d["value"] <= cfg.T
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
@@ -59,6 +67,28 @@ def test_gpu_count_must_match_the_launch():
                         "tiny_fp32", "--steps", "1", "--warmup", "0"], cwd=ROOT, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode != 0 and "--gpus 2" in r.stderr
+
+
+def test_roofline_objects_and_the_note_above_one():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_42_b200 import inputs
+    cfg = inputs.CONFIGS["v3_decode"]
+    up_f, up_b = bench.up_kernel_work(cfg, 158)
+    pk, _ = bench.peaks()
+    # a launch at exactly the HBM peak, then one faster than the copy peak
+    t = up_b / (pk["hbm_gbs"] * 1e9) * 1e3
+    roof, layer = bench.rooflines(cfg, 158, 2.2, {"experts_up": t}, False)
+    assert roof["bound"] == "hbm" and abs(roof["frac"] - 1.0) < 1e-9 and "note" not in roof
+    assert abs(roof["frac_nominal"] - pk["hbm_gbs"] / 8000.0) < 1e-9
+    roof, _ = bench.rooflines(cfg, 158, 2.2, {"experts_up": 0.9 * t}, False)
+    assert roof["frac"] > 1.0 and "note" in roof
+    assert layer["bound"] == "hbm" and 0 < layer["frac_nominal"] < layer["frac"]
+    # prefill is bound by the tensor cores
+    p = inputs.CONFIGS["v3_prefill"]
+    roof, layer = bench.rooflines(p, 256, 8.0, {"experts_up": 5.0}, True)
+    assert roof["bound"] == "tensor" and roof["peak_source"].endswith("(sustained)")
+    assert layer["bound"] == "tensor" and layer["frac_sustained"] > layer["frac"]
 
 
 def test_l2_note_states_how_the_timed_loop_meets_l2():
