@@ -16,7 +16,9 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "_lib", "libmoe.so")
+# The in-tree build; MOE_LIB_PATH names another build of the same library
+# (for example one compiled with different tile constants, to compare them).
+LIB_PATH = os.environ.get("MOE_LIB_PATH") or os.path.join(_PKG, "_lib", "libmoe.so")
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1

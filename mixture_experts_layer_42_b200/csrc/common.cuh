@@ -60,12 +60,16 @@ inline int act_bytes(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 
 constexpr int kFp8Block = 128;
 
 // Extra workspace regions of moe_forward_fp8, after the common layout.
+// (Activation scales are stored with their row stride, K/128, rounded up to
+// a multiple of 4 floats: see fp8_scale_stride.)
 struct Fp8Layout {
   size_t xq, xs;        // quantized x [T, D] e4m3, its scales [T, D/128] fp32
+  size_t xs_perm;       // x's scales in expert order [T*k, D/128]
   size_t hq, hs;        // quantized h [T*k, I], scales [T*k, I/128]
   size_t hsq, hss;      // the shared MLP's h [T, I_s], scales [T, I_s/128]
   size_t total;
 };
+inline int fp8_stride_host(int K) { return ((K / kFp8Block) + 3) & ~3; }
 
 // CTAs the router GEMM aims for (two per SM of a 148-SM B200).
 constexpr int kRouterTargetCtas = 296;
@@ -96,11 +100,12 @@ inline Fp8Layout fp8_layout(const moe_config& c, int64_t T, size_t base) {
     return o;
   };
   L.xq = take((size_t)T * D);
-  L.xs = take((size_t)T * (D / kFp8Block) * 4);
+  L.xs = take((size_t)T * fp8_stride_host((int)D) * 4);
+  L.xs_perm = take((size_t)T * k * fp8_stride_host((int)D) * 4);
   L.hq = take((size_t)T * k * I);
-  L.hs = take((size_t)T * k * (I / kFp8Block) * 4);
+  L.hs = take((size_t)T * k * fp8_stride_host((int)I) * 4);
   L.hsq = take((size_t)T * (Is > 0 ? Is : 1));
-  L.hss = take((size_t)T * (Is > 0 ? Is / kFp8Block : 1) * 4);
+  L.hss = take((size_t)T * (Is > 0 ? fp8_stride_host((int)Is) : 1) * 4);
   L.total = off;
   return L;
 }
@@ -248,19 +253,20 @@ struct Fp8Weights {
   const uint8_t *w1, *w3, *w2, *ws1, *ws3, *ws2;
   const float *s1, *s3, *s2, *ss1, *ss3, *ss2;
 };
-// Activation rows [R, K] (act) to e4m3 with one scale per 1 x 128 block.
+// Activation rows [R, K] (act) to e4m3 with one scale per 1 x 128 block;
+// the scales' row stride is sstride floats (<= 0: K/128).
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
-                              float* scale, cudaStream_t st);
+                              float* scale, int sstride, cudaStream_t st);
 // A matrix [R, C] (bf16 or fp32) to e4m3 with one scale per 128 x 128 block.
 cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
                                 float* scale, cudaStream_t st);
 // The FP8 expert GEMMs (gemm_fp8.cu): UP from the quantized x (routed rows
 // through src) into the quantized h, DOWN from it into y_perm and s (act).
 cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights& w,
-                               const uint8_t* xq, const float* xs, const int32_t* src,
-                               const int32_t* offsets, uint8_t* hq, float* hsc, uint8_t* hsq,
-                               float* hss, void* y_perm, void* s, uint32_t* err, int num_sms,
-                               cudaStream_t st);
+                               const uint8_t* xq, const float* xs, float* xs_perm,
+                               const int32_t* src, const int32_t* offsets, uint8_t* hq, float* hsc,
+                               uint8_t* hsq, float* hss, void* y_perm, void* s, uint32_t* err,
+                               int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
 // Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).

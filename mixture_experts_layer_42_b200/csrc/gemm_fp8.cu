@@ -34,19 +34,35 @@ namespace {
 using namespace tc;
 
 constexpr int QB = 128;                        // scale block edge; K per stage; weight rows per tile
-constexpr int NT = 64;                         // tokens per tile at most (MMA N)
-constexpr int FSTAGES = 4;
-constexpr int A_BYTES = NT * QB;               // 8 KB of token rows
+constexpr int NT = 32;                         // tokens per tile at most (MMA N)
+constexpr int A_BYTES = NT * QB;               // 4 KB of token rows
 constexpr int W_BYTES = QB * QB;               // 16 KB per weight tile
-constexpr int FSTAGE = A_BYTES + 2 * W_BYTES;  // UP: w1 and w3 tiles; DOWN uses one
+// Stages: UP carries the w1 and w3 tiles (36 KB, 5 stages), DOWN one w2 tile
+// (20 KB, 9 stages), so both keep ~160-180 KB of weights in flight per SM.
+template <bool UP> struct Ring {
+  static constexpr int STAGES = UP ? 5 : 9;
+  static constexpr int BYTES = A_BYTES + (UP ? 2 : 1) * W_BYTES;
+};
+constexpr int MAX_STAGES = 9;
+constexpr int RING_BYTES = 9 * (A_BYTES + W_BYTES);  // the larger of the two rings (184 KB)
+static_assert(5 * (A_BYTES + 2 * W_BYTES) <= RING_BYTES, "UP ring");
 constexpr int NTHREADS = 192;
 constexpr uint32_t FTMEM = 512;
 constexpr int MAXE = 1024;
 constexpr int MAX_KB = 64;                     // k-blocks per tile (K <= 8192)
-constexpr int NBUF_UP = 4;                     // TMEM buffers of 2 x NT columns
-constexpr int NBUF_DOWN = 8;                   // TMEM buffers of NT columns
-constexpr size_t FSMEM = 1024 + (size_t)FSTAGES * FSTAGE + 512 + 2 * (MAXE + 1) * 4 +
-                         (size_t)NT * MAX_KB * 4 + 4 * NT * 4;
+constexpr int NBUF_UP = 8;                     // TMEM buffers of 2 x NT columns
+constexpr int NBUF_DOWN = 16;                  // TMEM buffers of NT columns
+// The epilogue drains k-blocks KG at a time: one barrier wait (on the
+// group's last buffer: commits complete in order) and one tcgen05.wait::ld
+// per group instead of per k-block, so their latencies do not pace the
+// pipeline (one k-block at a time, the FP8 up-projection of a 32-expert
+// decode batch took longer than the bf16 one for half the bytes).
+constexpr int KG = 4;
+constexpr int SC_SLOT = NT * MAX_KB * 4;      // one tile's token scales (16 KB)
+// alignment slack, stages, barriers (512), P and off, 16 bytes to align the
+// scale slots, the two scale slots, the per-warp maxima
+constexpr size_t FSMEM = 1024 + (size_t)RING_BYTES + 512 + 2 * (MAXE + 1) * 4 + 16 +
+                         2 * (size_t)SC_SLOT + 4 * NT * 4;
 
 // kind::f8f6f4 instruction descriptor: fp32 accumulator, e4m3 A and B, both
 // K-major, M x N.
@@ -69,11 +85,17 @@ struct Fp8Args {
   // (UP: the quantized x, read by token through src; DOWN: the quantized h
   // in expert order), [1] the shared MLP's (UP: quantized x; DOWN: its h)
   CUtensorMap tmA[2];
+  // the same tensors for tile loads of contiguous rows (boxes of 16 and 32
+  // rows): every A but the routed UP's, whose rows are gathered by token
+  CUtensorMap tmAt[2][2];
   CUtensorMap tmW1[2];   // weights [E, N, K] uint8, box 128 x 128 x 1: w1 (UP) / w2 (DOWN); shared E = 1
   CUtensorMap tmW3[2];   // w3 / ws3 (UP)
   const float* ws1[2];   // weight scales [E, N/128, K/128] of tmW1
   const float* ws3[2];   // of tmW3
-  const float* asc[2];   // token rows' scales [rows, K/128]
+  // scales of the A rows [rows, K/128], in the A rows' order: routed UP the
+  // quantized x's scales permuted into expert order (gather_scales_kernel),
+  // so that a tile's are one contiguous run the producer copies in bulk
+  const float* asc[2];
   const int32_t* src;    // routed UP: the token of each expert-order row
   int a_rows[2];         // rows of the A tensors (an out-of-range row reads zeros)
   void* out[2];          // UP: quantized h [rows, N] uint8; DOWN: bf16 [rows, N]
@@ -128,6 +150,11 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
 
 __device__ __forceinline__ int round16(int r) { return (r + 15) & ~15; }
 
+// Row stride, in floats, of the activation scales inside the layer: K/128
+// rounded up to a multiple of 4, so every row starts 16-byte aligned and a
+// tile's rows can be copied in one bulk copy.
+__host__ __device__ __forceinline__ int scale_stride(int K) { return ((K / QB) + 3) & ~3; }
+
 // Smallest s with amax <= 448 * 2^s (0 for amax == 0): amax = m 2^e with
 // 0.5 <= m < 1, so s = e - 9, plus one when 2m > 1.75.
 __device__ __forceinline__ int block_exp(float amax) {
@@ -167,17 +194,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int NBUF = UP ? NBUF_UP : NBUF_DOWN;
   constexpr int BUF_COLS = UP ? 2 * NT : NT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + FSTAGES * FSTAGE);
+  constexpr int FSTAGES = Ring<UP>::STAGES;
+  constexpr int FSTAGE = Ring<UP>::BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + RING_BYTES);
   uint64_t* empty = full + FSTAGES;
   uint64_t* tfull = empty + FSTAGES;
   uint64_t* tempty = tfull + NBUF;
   uint64_t* drain = tempty + NBUF;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sfull = drain + 1;            // token-scale slots: copied in
+  uint64_t* sempty = sfull + 2;           //                    read by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* P = reinterpret_cast<int32_t*>(tiles + FSTAGES * FSTAGE + 512);
+  int32_t* P = reinterpret_cast<int32_t*>(tiles + RING_BYTES + 512);
   int32_t* off = P + MAXE + 1;
-  float* tsc = reinterpret_cast<float*>(off + MAXE + 1);  // [NT][MAX_KB] token scales of the tile
-  float* red = tsc + NT * MAX_KB;                         // [4][NT] per-warp maxima
+  // [2][rows][K/128] the token scales of a tile (two slots, copied in bulk
+  // by the producer a tile ahead), then [4][NT] per-warp maxima
+  float* tsc = reinterpret_cast<float*>(off + MAXE + 1 + 2);  // 16-byte aligned
+  float* red = tsc + 2 * NT * MAX_KB;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int E = g.E;
@@ -186,6 +219,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     if (lane == 0) {
       for (int s = 0; s < FSTAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
       for (int b = 0; b < NBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+      for (int b = 0; b < 2; ++b) { mbar_init(&sfull[b], 1); mbar_init(&sempty[b], 128); }
       mbar_init(drain, 1);
       *abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -245,14 +279,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // ---------------------------------------------------------------- TMA producer
     // lane 0: barriers and the weight tiles; lanes 0..n16/4-1: 4 token rows
     // each by tile::gather4
-    int s = 0, issued = 0;
+    int s = 0, issued = 0, scopies = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int i = blockIdx.x; i < S.total; i += gridDim.x) {
+    for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
       const Tile t = decode(S, i);
       const int kb_n = g.kdim[t.kind] / QB;
       const int n16 = round16(t.rows);
+      // the tile's token scales: t.rows contiguous rows of kb_n floats
+      {
+        int w = 1;
+        if (lane == 0) {
+          const int slot = lt & 1;
+          w = mbar_wait(&sempty[slot], ((lt >> 1) & 1) ^ 1, abort_flag, g.err) ? 1 : 0;
+          if (w) {
+            const int kbp = scale_stride(g.kdim[t.kind]);
+            const uint32_t bytes = (uint32_t)(t.rows * kbp * 4);
+            mbar_expect_tx(&sfull[slot], bytes);
+            bulk_load(tsc + slot * NT * MAX_KB, g.asc[t.kind] + (int64_t)t.row0 * kbp, bytes,
+                      &sfull[slot]);
+            ++scopies;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+      }
       const int n_g = n16 / 4;
+      // routed UP rows are tokens scattered over x: gathered four at a time;
+      // the others (expert-ordered h, token rows) are contiguous: one tile load
+      const bool gath = UP && t.kind == 0;
       const uint32_t tx = (uint32_t)(n16 * QB + (UP ? 2 : 1) * W_BYTES);
       int r[4];
 #pragma unroll
@@ -274,8 +328,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           tma_load_3d(sw, &g.tmW1[t.kind], &full[s], kb * QB, t.n0, t.e);
           if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], kb * QB, t.n0, t.e);
         }
+        if (!gath && lane == 0)   // contiguous rows: one tile load (rows past the end read zeros)
+          tma_load_2d(sa, &g.tmAt[t.kind][n16 > 16 ? 1 : 0], &full[s], kb * QB, t.row0);
         __syncwarp();
-        if (lane < n_g)
+        if (gath && lane < n_g)
           tma_gather4(sa + lane * (4 * QB), &g.tmA[t.kind], &full[s], kb * QB, r[0], r[1], r[2], r[3]);
         ++issued;
         if (++s == FSTAGES) { s = 0; ph ^= 1; }
@@ -286,6 +342,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       for (int j = 0; j < FSTAGES; ++j) {
         const int n = issued / FSTAGES + (j < issued % FSTAGES ? 1 : 0);
         if (n > 0) mbar_drain(&full[j], (uint32_t)((n - 1) & 1));
+      }
+      for (int j = 0; j < 2; ++j) {
+        const int n = scopies / 2 + (j < scopies % 2 ? 1 : 0);
+        if (n > 0) mbar_drain(&sfull[j], (uint32_t)((n - 1) & 1));
       }
     }
   } else if (warp == 1) {
@@ -328,66 +388,84 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     const int f = quad * 32 + lane;      // this thread's weight row (TMEM lane) in the tile
     const int et = threadIdx.x - 64;     // 0..127 among the epilogue threads
     int u = 0;
-    for (int i = blockIdx.x; i < S.total; i += gridDim.x) {
+    for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
       const Tile t = decode(S, i);
       const int kb_n = g.kdim[t.kind] / QB;
       const int n16 = round16(t.rows);
       bool ok = true;
-      // the tile's token scales for every k-block, into shared memory
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int q = et; q < NT * kb_n; q += 128) {
-        const int j = q / kb_n, kb = q % kb_n;
-        float v = 0.f;
-        if (j < t.rows) {
-          const int row = t.row0 + j;
-          const int a = (UP && t.kind == 0 && g.src != nullptr) ? g.src[row] : row;
-          v = g.asc[t.kind][(int64_t)a * kb_n + kb];
-        }
-        tsc[j * MAX_KB + kb] = v;
+      // the tile's token scales, copied in by the producer
+      const int slot = lt & 1;
+      {
+        int w = 1;
+        if (lane == 0) w = mbar_wait(&sfull[slot], (lt >> 1) & 1, abort_flag, g.err) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const float* sc = tsc + slot * NT * MAX_KB;   // [t.rows][kbp]
+      const int kbp = scale_stride(g.kdim[t.kind]);
       const int nbw = g.n_out[t.kind] / QB;
       const float* sw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
       const float* sw3 = UP ? g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n : nullptr;
       float sa[NT], sb[UP ? NT : 1];
 #pragma unroll
       for (int j = 0; j < NT; ++j) { sa[j] = 0.f; if (UP) sb[j] = 0.f; }
-      for (int kb = 0; kb < kb_n; ++kb, ++u) {
-        const int b = u % NBUF;
-        const uint32_t use = (uint32_t)(u / NBUF);
-        int w = 1;
-        if (lane == 0) w = mbar_wait(&tfull[b], use & 1, abort_flag, g.err) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+      for (int kb = 0; ok && kb < kb_n; kb += KG) {
+        const int gc = kb_n - kb < KG ? kb_n - kb : KG;   // k-blocks in this group
+        {
+          const int ul = u + gc - 1;
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&tfull[ul % NBUF], (uint32_t)(ul / NBUF) & 1, abort_flag, g.err) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        }
         tc_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * BUF_COLS);
-        const float c1 = __ldg(sw1 + kb);
-        const float c3 = UP ? __ldg(sw3 + kb) : 0.f;
+        float c1[KG], c3[KG];
+#pragma unroll
+        for (int q = 0; q < KG; ++q) {
+          c1[q] = q < gc ? __ldg(sw1 + kb + q) : 0.f;
+          c3[q] = (UP && q < gc) ? __ldg(sw3 + kb + q) : 0.f;
+        }
 #pragma unroll
         for (int j0 = 0; j0 < NT; j0 += 16) {
           if (j0 < n16) {
-            uint32_t ra[16], rb[16];
-            tmem_ld16(tb + j0, ra);
-            if (UP) tmem_ld16(tb + NT + j0, rb);
+            uint32_t ra[KG][16], rb[KG][UP ? 16 : 1];
+#pragma unroll
+            for (int q = 0; q < KG; ++q) {
+              if (q < gc) {
+                const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                    (uint32_t)(((u + q) % NBUF) * BUF_COLS);
+                tmem_ld16(tb + j0, ra[q]);
+                if (UP) tmem_ld16(tb + NT + j0, *reinterpret_cast<uint32_t(*)[16]>(rb[q]));
+              }
+            }
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float xs = tsc[(j0 + q) * MAX_KB + kb];
-              sa[j0 + q] = fmaf(__uint_as_float(ra[q]), c1 * xs, sa[j0 + q]);
-              if (UP) sb[j0 + q] = fmaf(__uint_as_float(rb[q]), c3 * xs, sb[j0 + q]);
+            for (int q = 0; q < KG; ++q) {
+              if (q < gc) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                  // rows past the tile's tokens: their products are zero, and
+                  // the slot holds no scale for them
+                  const float xs = (j0 + c < t.rows) ? sc[(j0 + c) * kbp + kb + q] : 0.f;
+                  sa[j0 + c] = fmaf(__uint_as_float(ra[q][c]), c1[q] * xs, sa[j0 + c]);
+                  if (UP) sb[j0 + c] = fmaf(__uint_as_float(rb[q][c]), c3[q] * xs, sb[j0 + c]);
+                }
+              }
             }
           }
         }
         tc_fence_before();
-        mbar_arrive(&tempty[b]);
+        for (int q = 0; q < gc; ++q) mbar_arrive(&tempty[(u + q) % NBUF]);
+        u += gc;
       }
-      // one decision for all four warps: stop if any of them gave up
+      // one decision for all four warps: stop if any of them gave up; the
+      // scale slot is free once every epilogue thread is past its last read
       if (epi_sync_any(!ok)) break;
+      mbar_arrive(&sempty[slot]);
       if (UP) {
         // h = silu(a) * b, quantized per token over this tile's 128 features
         // (one 1 x 128 block of h's row)
         uint8_t* hq = reinterpret_cast<uint8_t*>(g.out[t.kind]);
         float* hs = g.out_scale[t.kind];
-        const int nbh = g.n_out[t.kind] / QB;
+        const int nbh = scale_stride(g.n_out[t.kind]);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           if (j >= n16) break;
@@ -433,7 +511,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
 template <typename T>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int64_t R, int K,
                                                          uint8_t* __restrict__ q,
-                                                         float* __restrict__ scale) {
+                                                         float* __restrict__ scale, int sstride) {
   const int kbn = K / QB;
   const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
@@ -452,7 +530,21 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
 #pragma unroll
   for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(ldexpf(v[i], -se)) << (8 * i);
   reinterpret_cast<uint32_t*>(q + r * K + kb * QB)[lane] = packed;
-  if (lane == 0) scale[r * kbn + kb] = ldexpf(1.f, se);
+  if (lane == 0) scale[r * sstride + kb] = ldexpf(1.f, se);
+}
+
+// The quantized x's scales in expert order: row p takes token src[p]'s
+// (rows at or past offsets[E] are not read by the experts and are skipped).
+__global__ void __launch_bounds__(256) gather_scales_kernel(const float* __restrict__ xs,
+                                                            const int32_t* __restrict__ src,
+                                                            const int32_t* __restrict__ offsets,
+                                                            int E, int64_t Tk, int sstride,
+                                                            float* __restrict__ xs_perm) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t p = i / sstride;
+  const int kb = (int)(i % sstride);
+  if (p >= Tk || p >= offsets[E]) return;
+  xs_perm[i] = xs[(int64_t)src[p] * sstride + kb];
 }
 
 // A bf16 / fp32 matrix [R, C] to e4m3 with one power-of-two scale per
@@ -500,6 +592,18 @@ bool map_u8_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool map_u8_tile(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K};
+  cuuint32_t box[2] = {QB, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uint64_t K) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -515,16 +619,20 @@ bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uin
 }  // namespace
 
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
-                              float* scale, cudaStream_t st) {
+                              float* scale, int sstride, cudaStream_t st) {
   const int64_t warps = R * (K / QB);
   if (warps == 0) return cudaSuccess;
+  if (sstride <= 0) sstride = K / QB;
   const unsigned blocks = (unsigned)ceil_div<int64_t>(warps * 32, 256);
   if (c.dtype == MOE_DT_BF16)
-    quant_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)a, R, K, q, scale);
+    quant_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)a, R, K, q, scale,
+                                                              sstride);
   else
-    quant_rows_kernel<float><<<blocks, 256, 0, st>>>((const float*)a, R, K, q, scale);
+    quant_rows_kernel<float><<<blocks, 256, 0, st>>>((const float*)a, R, K, q, scale, sstride);
   return cudaGetLastError();
 }
+
+int fp8_scale_stride(int K) { return scale_stride(K); }
 
 cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
                                 float* scale, cudaStream_t st) {
@@ -540,14 +648,20 @@ cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint
 // by token through src, shared rows directly) and writes the quantized h and
 // hs; DOWN reads them and writes y_perm and s (bf16).
 cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights& w,
-                               const uint8_t* xq, const float* xs, const int32_t* src,
-                               const int32_t* offsets, uint8_t* hq, float* hsc, uint8_t* hsq,
-                               float* hss, void* y_perm, void* s, uint32_t* err, int num_sms,
-                               cudaStream_t st) {
+                               const uint8_t* xq, const float* xs, float* xs_perm,
+                               const int32_t* src, const int32_t* offsets, uint8_t* hq, float* hsc,
+                               uint8_t* hsq, float* hss, void* y_perm, void* s, uint32_t* err,
+                               int num_sms, cudaStream_t st) {
   const int E = c.n_routed, D = c.dim, I = c.moe_inter, Is = c.shared_inter;
   const int64_t Tk = T * c.topk;
   const bool sh = Is > 0;
   cudaError_t e;
+  {
+    const int ss = scale_stride(D);
+    gather_scales_kernel<<<(unsigned)ceil_div<int64_t>(Tk * ss, 256), 256, 0, st>>>(
+        xs, src, offsets, E, Tk, ss, xs_perm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   for (int pass = 0; pass < 2; ++pass) {
     const bool up = pass == 0;
     Fp8Args g;
@@ -556,7 +670,7 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
     if (up) {
       if (!map_u8_rows(&g.tmA[0], xq, (uint64_t)T, (uint64_t)D)) return cudaErrorInvalidValue;
       g.a_rows[0] = (int)T;
-      g.asc[0] = xs;
+      g.asc[0] = xs_perm;
       g.src = src;
       if (!map_u8_weights(&g.tmW1[0], w.w1, E, I, D)) return cudaErrorInvalidValue;
       if (!map_u8_weights(&g.tmW3[0], w.w3, E, I, D)) return cudaErrorInvalidValue;
@@ -589,6 +703,22 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
         if (!map_u8_weights(&g.tmW1[1], w.ws2, 1, D, Is)) return cudaErrorInvalidValue;
         g.ws1[1] = w.ss2;
         g.out[1] = s;
+      }
+    }
+    // tile-load maps of the A tensors (boxes of 16 and 32 rows)
+    {
+      const void* a0p = up ? (const void*)xq : (const void*)hq;
+      const uint64_t r0 = up ? (uint64_t)T : (uint64_t)Tk, kk0 = up ? (uint64_t)D : (uint64_t)I;
+      for (int b = 0; b < 2; ++b)
+        if (!map_u8_tile(&g.tmAt[0][b], a0p, r0, kk0, 16u << b)) return cudaErrorInvalidValue;
+      if (sh) {
+        const void* a1p = up ? (const void*)xq : (const void*)hsq;
+        const uint64_t kk1 = up ? (uint64_t)D : (uint64_t)Is;
+        for (int b = 0; b < 2; ++b)
+          if (!map_u8_tile(&g.tmAt[1][b], a1p, (uint64_t)T, kk1, 16u << b)) return cudaErrorInvalidValue;
+      } else {
+        g.tmAt[1][0] = g.tmAt[0][0];
+        g.tmAt[1][1] = g.tmAt[0][1];
       }
     }
     if (!sh) {  // no shared group: its maps are never used, keep them valid

@@ -20,10 +20,18 @@
 // (one 4D TMA box over both tensors when their distance allows, else two
 // boxes), so accumulator columns j and 128+j hold a and b of the same feature.
 //
+// The up-projection's routed A rows come either from an expert-contiguous
+// copy of x (one tile load per stage) or straight from x through the
+// dispatch's src (tile::gather4: each lane of the TMA warp brings 4 rows, 32
+// copies per 128-row stage). The gathers bound a 128-row stage by the TMA's
+// copy rate, so the layer gathers only for decode-sized batches, whose
+// experts run one swapped tile of a few rows (see below).
+//
 // An expert's last, partial m-tile loads its A rows through a copy of the A
 // tensor map whose row extent ends at the expert's last row (one per expert,
 // written by build_row_maps_kernel before the launch): TMA fills the rows
-// past it with zeros instead of the next expert's rows. The results are the
+// past it with zeros instead of the next expert's rows. Gathered rows past
+// the expert get an out-of-range row and read zeros too. The results are the
 // same (those rows are never stored), but zero operands draw less power, and
 // under the board's power cap that buys clock.
 //

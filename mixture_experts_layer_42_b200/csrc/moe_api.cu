@@ -467,7 +467,7 @@ moe_status moe_quantize_fp8(const moe_config* cfg, const void* a, int64_t rows, 
   moe_status st = bind_device(s, a);
   if (st != MOE_OK) return st;
   if (block_rows == 1)
-    return cuda_status(launch_quant_rows(*cfg, a, rows, (int)cols, static_cast<uint8_t*>(q), scales, s));
+    return cuda_status(launch_quant_rows(*cfg, a, rows, (int)cols, static_cast<uint8_t*>(q), scales, 0, s));
   return cuda_status(launch_quant_blocks(cfg->dtype == MOE_DT_BF16, a, rows, (int)cols,
                                          static_cast<uint8_t*>(q), scales, s));
 }
@@ -526,14 +526,16 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
   // x to e4m3 once per step (its kernel is timed with the up-projection)
   uint8_t* xq = at<uint8_t>(ws, F.xq);
   float* xs = at<float>(ws, F.xs);
-  if (launch_quant_rows(c, x, T, c.dim, xq, xs, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_quant_rows(c, x, T, c.dim, xq, xs, fp8_stride_host(c.dim), s) != cudaSuccess)
+    return MOE_ERR_CUDA;
   Fp8Weights fw{static_cast<const uint8_t*>(w->w1), static_cast<const uint8_t*>(w->w3),
                 static_cast<const uint8_t*>(w->w2), static_cast<const uint8_t*>(w->ws1),
                 static_cast<const uint8_t*>(w->ws3), static_cast<const uint8_t*>(w->ws2),
                 w->w1_scale, w->w3_scale, w->w2_scale, w->ws1_scale, w->ws3_scale, w->ws2_scale};
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
-  if (launch_grouped_fp8(c, T, fw, xq, xs, src, offsets, at<uint8_t>(ws, F.hq), at<float>(ws, F.hs),
+  if (launch_grouped_fp8(c, T, fw, xq, xs, at<float>(ws, F.xs_perm), src, offsets,
+                         at<uint8_t>(ws, F.hq), at<float>(ws, F.hs),
                          at<uint8_t>(ws, F.hsq), at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf,
                          err, num_sms_current(), s) != cudaSuccess)
     return MOE_ERR_CUDA;

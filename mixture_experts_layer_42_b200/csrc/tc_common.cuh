@@ -139,6 +139,16 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tm, ui
       : "memory");
 }
 
+// Contiguous bytes (a multiple of 16, both addresses 16-byte aligned) from
+// global to shared memory, completing on an mbarrier (non-tensor bulk copy).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Make a tensor map written to global memory through the generic proxy
 // (tensormap.cp_fenceproxy ... release) visible to this thread's TMA loads.
 __device__ __forceinline__ void tmap_acquire(const void* map) {

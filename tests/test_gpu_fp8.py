@@ -61,18 +61,25 @@ class Fp8Layer:
                                 self.q["w1"][1], self.q["w3"][1], self.q["w2"][1],
                                 *(self.q[n][0] if n in self.q else None for n in ("ws1", "ws3", "ws2")),
                                 *(self.q[n][1] if n in self.q else None for n in ("ws1", "ws3", "ws2")))
-        self.deq = {n: O.dequantize_blocks(codes(q), s.cpu().numpy().astype(np.float64), 128, 128)
-                    for n, (q, s) in self.q.items()}
         self.shape = dict(w1=(E, I, D), w3=(E, I, D), w2=(E, D, I))
 
+    def _deq(self, name, e=None):
+        """Dequantized weights (exact: code times its block's power of two);
+        for routed experts one expert at a time, as the oracle asks for them."""
+        q, s = self.q[name]
+        if e is not None:
+            _, n, k = self.shape[name]
+            q = q[e * n:(e + 1) * n]
+            s = s[e * n // 128:(e + 1) * n // 128]
+        return O.dequantize_blocks(codes(q), s.cpu().numpy().astype(np.float64), 128, 128)
+
     def experts(self):
-        d = {n: self.deq[n].reshape(self.shape[n]) for n in ("w1", "w3", "w2")}
-        return lambda e: (d["w1"][e], d["w3"][e], d["w2"][e])
+        return lambda e: tuple(self._deq(n, e) for n in ("w1", "w3", "w2"))
 
     def shared(self):
-        if "ws1" not in self.deq:
+        if "ws1" not in self.q:
             return None
-        return self.deq["ws1"], self.deq["ws3"], self.deq["ws2"]
+        return tuple(self._deq(n) for n in ("ws1", "ws3", "ws2"))
 
     def forward(self):
         L, cfg = self.L, self.L.cfg
