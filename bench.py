@@ -19,8 +19,8 @@ tokens of all ranks over the slowest rank's device time.
 Printed (rank 0, one JSON line): tokens/s from CUDA events on the launching
 stream; e2e tokens/s through the same C call with x copied in from pinned host
 memory and y copied back every step; the roofline of the dominant kernel from
-per-kernel CUDA events recorded inside the timed region (on one step in ten);
-the layer roofline; the CPU oracle's rate on a bounded token sample (N=1
+per-kernel CUDA events recorded in a separate untimed pass after the timed
+loop (which records no other event); the layer roofline; the CPU oracle's rate on a bounded token sample (N=1
 only); SM clocks sampled during the run. At N=1 the line also carries
 `workloads`: the same device-timed measurements for the other bf16 workloads
 (V3 prefill, the Zipf-skewed prefill, the softmax layer), each timed for about
@@ -456,9 +456,12 @@ class Setup:
 def device_timed(S, D, steps, warmup, uuid, clocks_on):
     """Time `steps` forwards on the device after `warmup` untimed ones:
     barrier + synchronize on both sides, CUDA events on the launching stream,
-    max over ranks. Per-kernel events are recorded on one step in ten (at
-    least one step) inside the same timed loop. Returns (ms, kernels_ms per
-    launch, steps recorded, every, clocks)."""
+    max over ranks; the timed loop records no other event. The per-kernel
+    times come from a separate, untimed pass right after it (a tenth of the
+    steps, 2 to 20), whose forwards record an event between every two kernels
+    and so run all their kernels on the one stream (the shared expert's
+    up-projection inside the routed experts' launch). Returns (ms, kernels_ms
+    per launch, kernels_ms_steps, clocks)."""
     M = S.M
     clocks = Clocks() if clocks_on else None
     for _ in range(warmup):
@@ -467,8 +470,6 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     D.barrier()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    every = max(10, steps // 20) if steps >= 10 else steps
-    M.moe_stage_timing_begin_every((steps + every - 1) // every, every)
     wall0 = time.time()
     ev0.record(S.stream)
     for _ in range(steps):
@@ -478,12 +479,19 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     wall1 = time.time()
     D.barrier()
     torch.cuda.synchronize()
-    n_rec, stage_ms = M.moe_stage_timing_end()
     ms = D.max(ev0.elapsed_time(ev1))
+    n_pass = min(20, max(2, steps // 10))
+    M.moe_stage_timing_begin(n_pass)
+    for _ in range(n_pass):
+        S.step()
+    torch.cuda.synchronize()
+    n_rec, stage_ms = M.moe_stage_timing_end()
     if M.moe_check_error(S.ws, S.stream) != M.MOE_OK:
         raise RuntimeError(f"{S.cfg.name}: device error word set during the timed loop")
     ck = clocks.stop(wall0, wall1, uuid) if clocks else None
-    return ms, {k: v / max(n_rec, 1) for k, v in stage_ms.items()}, n_rec, every, ck
+    rec = {"recorded": n_rec, "pass": "separate, untimed, after the timed loop; each recorded "
+                                      "forward runs its kernels on one stream"}
+    return ms, {k: v / max(n_rec, 1) for k, v in stage_ms.items()}, rec, ck
 
 
 def rooflines(cfg, n_active, ms_step, per_kernel_ms, long_run):
@@ -540,7 +548,7 @@ def other_workload(name, a, D, dev, uuid, shared_weights):
     torch.cuda.synchronize()
     est = t0.elapsed_time(t1) / 3
     steps = int(min(2000, max(a.steps, 1000.0 / max(est, 1e-3))))
-    ms, per_kernel_ms, n_rec, every, ck = device_timed(S, D, steps, a.warmup, uuid, True)
+    ms, per_kernel_ms, rec, ck = device_timed(S, D, steps, a.warmup, uuid, True)
     ms_step = ms / steps
     roof, layer = rooflines(cfg, n_active, ms_step, per_kernel_ms, ms > 1000.0)
     del S
@@ -548,7 +556,7 @@ def other_workload(name, a, D, dev, uuid, shared_weights):
             "steps": steps, "warmup": a.warmup, "ms_per_step": ms_step,
             "value": cfg.T * steps / (ms / 1e3), "unit": UNIT, "roofline": roof,
             "layer_roofline": layer, "kernels_ms": per_kernel_ms,
-            "kernels_ms_steps": {"recorded": n_rec, "every": every},
+            "kernels_ms_steps": rec,
             "dominant_kernel": max(per_kernel_ms, key=per_kernel_ms.get), "routing": routing,
             "clocks": ck}
 
@@ -571,7 +579,7 @@ def ours_arm(a, D):
         pass
 
     # ------------------------------------------------------------ device-timed loop
-    ms, per_kernel_ms, n_rec, every, ck = device_timed(S, D, a.steps, a.warmup, uuid, D.rank == 0)
+    ms, per_kernel_ms, rec, ck = device_timed(S, D, a.steps, a.warmup, uuid, D.rank == 0)
 
     # ------------------------------------------------------------ end to end (host buffers)
     # Each step copies its x in from pinned host memory and its y back out.
@@ -672,7 +680,7 @@ def ours_arm(a, D):
             "gpu_launches": launches * a.steps * N,
             "roofline": roof,
             "layer_roofline": layer,
-            "kernels_ms": per_kernel_ms, "kernels_ms_steps": {"recorded": n_rec, "every": every},
+            "kernels_ms": per_kernel_ms, "kernels_ms_steps": rec,
             "dominant_kernel": max(per_kernel_ms, key=per_kernel_ms.get), "active_experts": n_active,
             "routing": routing,
             "cpu_baseline": cpu, "clocks": ck,

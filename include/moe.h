@@ -173,7 +173,12 @@ MOE_API moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_p
  * permuted copy of x is made. Larger bf16 batches, and the CTA-pair expert
  * kernel, read an expert-contiguous copy that dispatch writes into the
  * workspace's y_perm region (free until the down-projection writes it): on
- * B200 the copy is the faster of the two for 128-row tiles. */
+ * B200 the copy is the faster of the two for 128-row tiles. On the default
+ * one-CTA tensor-core kernel the up-projection is launched as a programmatic
+ * dependent of the dispatch's last kernel (cudaLaunchKernelEx with
+ * programmatic stream serialization): its CTAs start, and take any shared-
+ * expert tiles, while that kernel finishes, and wait for it (griddepcontrol)
+ * before their first routed tile. */
 MOE_API moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
                        const float* bias, const void* w1, const void* w3, const void* w2,
                        const void* ws1, const void* ws3, const void* ws2, void* y,
@@ -277,7 +282,7 @@ MOE_API const char* moe_status_string(moe_status st);
 /* Number of kernels moe_forward launches for this config with the expert
  * kernel currently selected (moe_select_expert_kernel), for accounting: 9
  * for a bf16 layer on the default one-CTA tensor-core kernel (the expert GEMMs
- * follow one kernel that writes their per-expert A maps), 8 otherwise. */
+ * use one kernel that writes their per-expert A maps), 8 otherwise. */
 MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
 
 /* moe_gate without a workspace. The pages have no counterpart of this call:
@@ -323,10 +328,12 @@ MOE_API moe_status moe_gate_noalloc_check_error(const void* x, void* stream);
  * moe_forward_launch_count() kernels. moe_stage_timing_end(ms, n) disarms,
  * waits for the recorded events and writes to ms[i] the total milliseconds
  * kernel i (launch order: router logits, router select, dispatch rank,
- * dispatch scan, dispatch positions, experts up -- with the per-expert map
- * kernel before it, when there is one --, experts down, combine) took
- * over the recorded calls, for i < n <= 8; it returns the number of calls
- * recorded, or a negative moe_status. Single-threaded use only. */
+ * dispatch scan, dispatch positions -- with the per-expert map kernel before
+ * it, when there is one --, experts up, experts down, combine) took over the
+ * recorded calls, for i < n <= 8; it returns the number of calls recorded, or
+ * a negative moe_status. A recorded call launches its up-projection as an
+ * ordinary launch (not as a programmatic dependent of the dispatch), so that
+ * each interval holds one kernel. Single-threaded use only. */
 MOE_API moe_status moe_stage_timing_begin(int32_t max_calls);
 MOE_API int32_t moe_stage_timing_end(float* ms, int32_t n);
 

@@ -30,16 +30,27 @@ combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ pos,
   float acc[VE];
 #pragma unroll
   for (int q = 0; q < VE; ++q) acc[q] = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const int p = p_s[j];
-    if (p < 0) continue;
-    Vec16<T> r;
-    r.raw = reinterpret_cast<const uint4*>(y_perm + (int64_t)p * D)[v];
-    float f[VE];
-    r.to_float(f);
-    const float w = w_s[j];
+  // the token's rows, 8 at a time: all loads issued before the first add
+  // (more bytes in flight per thread), then added in slot order
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    uint4 raw[8];
 #pragma unroll
-    for (int q = 0; q < VE; ++q) acc[q] = fmaf(w, f[q], acc[q]);
+    for (int u = 0; u < 8; ++u) {
+      const int p = j0 + u < k ? p_s[j0 + u] : -1;
+      raw[u] = p >= 0 ? reinterpret_cast<const uint4*>(y_perm + (int64_t)p * D)[v]
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (j0 + u >= k || p_s[j0 + u] < 0) continue;
+      Vec16<T> r;
+      r.raw = raw[u];
+      float f[VE];
+      r.to_float(f);
+      const float w = w_s[j0 + u];
+#pragma unroll
+      for (int q = 0; q < VE; ++q) acc[q] = fmaf(w, f[q], acc[q]);
+    }
   }
   if (s) {
     Vec16<T> r;

@@ -213,6 +213,10 @@ struct GroupedArgs {
 // stage timing on (see moe_stage_timing_begin); a no-op otherwise. Every
 // launcher calls it right after each kernel it launches.
 void stage_mark(cudaStream_t st);
+// Whether the stage timer is recording the current forward call.
+bool stage_timing_active();
+// SMs of the current device (cached per device).
+int num_sms_current();
 
 // Router: logits (tensor cores for bf16 unless `simt`, else CUDA cores) into
 // `part` with at most `splits` k splits, then selection into weights / idx.
@@ -232,10 +236,31 @@ size_t gate_scratch_floats();
 cudaError_t gate_scratch_current_device(float** scratch, uint32_t** err);
 
 // x_perm may be null: then only counts, offsets, src and pos are written.
+// zero_ctr (nullable): an int the scan kernel sets to 0 (the up-projection's
+// tile counter, when the experts follow in the same stream).
 cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
                             int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                             void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,
                             uint32_t* err, cudaStream_t st);
+// The dispatch in its two halves: the sort (counts, offsets, each pair's
+// rank within its chunk), then the placement (pos, src and, when x_perm is
+// given, the permuted copy of x). The placement lets a programmatic dependent
+// launch start at once (it must wait for the grid before reading src or x_perm).
+cudaError_t launch_dispatch_sort(const moe_config& c, int64_t T, const int32_t* idx,
+                                 int32_t* counts, int32_t* offsets, int32_t* chunk_hist,
+                                 int32_t* pos_local, int n_chunks, uint32_t* err, cudaStream_t st);
+struct DispatchPlace {
+  const moe_config* c;
+  int64_t T;
+  const int32_t* idx;
+  const void* x;
+  const int32_t* chunk_hist;
+  const int32_t* pos_local;
+  int32_t* pos;
+  int32_t* src;
+  void* x_perm;
+};
+cudaError_t launch_dispatch_place(const DispatchPlace& p, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, const int32_t* pos,
                            const float* weights, const void* s, void* y, cudaStream_t st);
 // Expert parallelism: one rank's fp32 share of y (pairs routed to its
@@ -285,11 +310,12 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, const void* gx,
                               const int32_t* src, int64_t gT, const void* row_maps, int* tile_ctr,
-                              uint32_t* err, int num_sms, cudaStream_t st);
+                              uint32_t* err, int num_sms, cudaStream_t st, bool pdl);
 // Before the one-CTA expert GEMMs: per-expert copies of the down-projection's
 // A map over h [Tk, I] (at maps + E) and, when a_up is given, of the
 // up-projection's over a_up [Tk, D] (at maps), each with its row extent cut
-// at the expert's end; zeroes the up-projection's tile counter.
+// at the expert's end; zeroes the up-projection's tile counter. Reads only
+// the offsets (a_up's rows need not be written yet).
 cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, int D,
                             const int32_t* offsets, int E, void* maps, int* up_tile_ctr,
                             cudaStream_t st);

@@ -46,6 +46,8 @@
 // what it has in flight, frees TMEM and returns.
 #include "tc_common.cuh"
 
+#include <utility>
+
 namespace moe {
 
 namespace {
@@ -82,9 +84,14 @@ struct Sched {
   int E, nt0, nt1, mt_sh, routed, total, t_shared, bn_out;
 };
 
+// Tile i: the shared expert's tiles come first (they need only x, so the
+// up-projection can run them while the dispatch that feeds the routed tiles
+// is still finishing), then the routed experts' tiles.
 __device__ __forceinline__ Tile decode(const Sched& S, int i) {
   Tile t;
-  if (i < S.routed) {
+  const int n_sh = S.total - S.routed;
+  if (i >= n_sh) {
+    i -= n_sh;
     const int q = i / S.nt0;
     int lo = 0, hi = S.E;  // the e with P[e] <= q < P[e+1]
     while (hi - lo > 1) {
@@ -102,7 +109,7 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
     t.n0 = nt * S.bn_out;
     t.only = mt == 1;
   } else {
-    const int l = i - S.routed;
+    const int l = i;
     const int nt = l / S.mt_sh, m = l % S.mt_sh;
     t.kind = 1;
     t.e = 0;
@@ -237,6 +244,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool ok = true;
+    bool dep_done = false;
     TileQueue Q;
     const bool dyn = g.tile_ctr != nullptr;
     // the next tile is claimed a few k-blocks before the current one ends,
@@ -263,6 +271,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       }
       if (i >= S.total) break;
       const Tile t = decode(S, i);
+      if (t.kind == 0 && !dep_done) {
+        // the routed rows (their copy or src), their maps: written by the
+        // kernels this launch may have started alongside (programmatic
+        // dependent launch); returns at once otherwise
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        dep_done = true;
+      }
       const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
       const int kb_claim = kb_n > 4 ? kb_n - 4 : 0;
       const bool swap = swap_tail(t, g);
@@ -567,6 +582,26 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
 
 }  // namespace
 
+// A launch on `st`, as a programmatic dependent of the kernel before it in the
+// stream when `pdl` (it may start once that kernel's CTAs have all executed
+// griddepcontrol.launch_dependents, and must griddepcontrol.wait before it
+// reads that kernel's output), else an ordinary launch.
+template <typename... Params, typename... Args>
+static cudaError_t launch_k(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Test hook state (moe_debug_stall_pipeline).
 static int g_stall = STALL_NONE;
 void set_pipeline_stall(int which) { g_stall = which; }
@@ -598,7 +633,7 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
                               const void* b3_1, int n0, int k0, int n1, int k1, void* out0,
                               void* out1, const int32_t* offsets, const void* gx,
                               const int32_t* src, int64_t gT, const void* row_maps, int* tile_ctr,
-                              uint32_t* err, int num_sms, cudaStream_t st) {
+                              uint32_t* err, int num_sms, cudaStream_t st, bool pdl) {
   TcArgs g;
   memset(&g, 0, sizeof(g));
   const bool pair = kind == TC_PAIR;
@@ -695,12 +730,14 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
     e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    grouped_tc_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(g);
+    e = launch_k(pdl, grouped_tc_kernel<true>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
+    if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(grouped_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    grouped_tc_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(g);
+    e = launch_k(pdl, grouped_tc_kernel<false>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
+    if (e != cudaSuccess) return e;
   }
   stage_mark(st);
   return cudaGetLastError();

@@ -51,6 +51,8 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
 }
 
+}  // namespace
+
 int num_sms_current() {
   static int cached[64] = {0};
   int dev = 0;
@@ -64,6 +66,8 @@ int num_sms_current() {
   }
   return cached[dev];
 }
+
+namespace {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -93,12 +97,18 @@ moe_status bind_device(cudaStream_t s, const void* ptr) {
 }
 
 // The expert GEMMs. The routed A rows come from x_perm (an expert-contiguous
-// copy of x) or, when x_perm is null, are gathered from x through src.
+// copy of x) or, when x_perm is null, are gathered from x through src. With
+// `place`, the dispatch's placement (pos, src, the copy) is launched here,
+// after the row maps (which need only the offsets) and right before the
+// up-projection, which then starts as a programmatic dependent of it (its
+// prologue and any shared-expert tiles, which come first and need only x, run
+// while the placement finishes; its producer waits for the placement's grid
+// before the first routed tile).
 moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* src,
                        const int32_t* offsets, const void* w1, const void* w3, const void* w2,
                        const void* x, const void* ws1, const void* ws3, const void* ws2,
                        void* y_perm, void* s, void* h, void* hs, void* row_maps, uint32_t* err,
-                       cudaStream_t st) {
+                       cudaStream_t st, const DispatchPlace* place = nullptr) {
   const int64_t Tk = T * c.topk;
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
@@ -120,17 +130,23 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
       e = launch_row_maps(h, Tk, c.moe_inter, x_perm, c.dim, offsets, c.n_routed, row_maps, ctr, st);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
+    if (place != nullptr && launch_dispatch_place(*place, num_sms_current(), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // (not while the stage timer records events between the launches)
+    const bool pdl = place != nullptr && kind == TC_ROWS && !stage_timing_active();
     e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                           c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets, x,
                           x_perm ? nullptr : src, T, kind == TC_ROWS ? row_maps : nullptr, ctr, err,
-                          num_sms_current(), st);
+                          num_sms_current(), st, pdl);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
                           c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, nullptr,
                           nullptr, 0, kind == TC_ROWS ? maps_down : nullptr, nullptr, err,
-                          num_sms_current(), st);
+                          num_sms_current(), st, false);
     return cuda_status(e);
   }
+  if (place != nullptr && launch_dispatch_place(*place, num_sms_current(), st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   GroupedArgs g;
   memset(&g, 0, sizeof(g));
   g.offsets = offsets;
@@ -203,6 +219,8 @@ bool fp8_shapes_ok(const moe_config& c) {
 }
 
 }  // namespace
+
+bool stage_timing_active() { return g_timing.on && g_timing.in_forward; }
 
 void stage_mark(cudaStream_t st) {
   StageTiming& T = g_timing;
@@ -374,15 +392,17 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   const bool copy_rows = c.dtype == MOE_DT_BF16 &&
                          (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR || big);
   void* x_perm = copy_rows ? at<void>(ws, L.y_perm) : nullptr;
-  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, src, pos, x_perm,
-                      at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
-                      s) != cudaSuccess)
+  if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
+                           at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks,
+                           err, s) != cudaSuccess)
     return MOE_ERR_CUDA;
+  const DispatchPlace place{&c, T, idx, x, at<int32_t>(ws, L.chunk_hist),
+                            at<int32_t>(ws, L.pos_local), pos, src, x_perm};
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
   st = run_experts(c, T, x_perm, src, offsets, w1, w3, w2, x, ws1, ws3, ws2,
                    at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
-                   at<void>(ws, L.row_maps), err, s);
+                   at<void>(ws, L.row_maps), err, s, &place);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
 }
@@ -417,6 +437,12 @@ moe_status moe_forward_ep(const moe_config* cfg, int64_t T, int32_t expert_begin
   float* weights = weights_out ? weights_out : at<float>(ws, L.weights);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, L.idx);
   uint32_t* err = at<uint32_t>(ws, L.header);
+  // this rank's experts are a contiguous run of the expert order: the
+  // grouped GEMMs see them as a layer of n_local experts whose offsets start
+  // at expert_begin's, and the shared MLP as one of width shared_local
+  moe_config lc = c;
+  lc.n_routed = expert_end - expert_begin;
+  lc.shared_inter = shared_local;
   // every rank routes every token over all experts (the gate is replicated)
   if (launch_router(c, T, x, w_router, bias, weights, idx, at<float>(ws, L.router_part),
                     L.router_splits, g_expert_kernel == MOE_EXPERT_KERNEL_SIMT, num_sms_current(),
@@ -428,21 +454,17 @@ moe_status moe_forward_ep(const moe_config* cfg, int64_t T, int32_t expert_begin
   // gathered rows or a permuted copy, by the same rule as moe_forward
   const bool big = T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed;
   void* x_perm = (c.dtype == MOE_DT_BF16 && big) ? at<void>(ws, L.y_perm) : nullptr;
-  if (launch_dispatch(c, T, idx, x, at<int32_t>(ws, L.counts), offsets, src, pos, x_perm,
-                      at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
-                      s) != cudaSuccess)
+  if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
+                           at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks,
+                           err, s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // this rank's experts are a contiguous run of the expert order: the
-  // grouped GEMMs see them as a layer of n_local experts whose offsets start
-  // at expert_begin's, and the shared MLP as one of width shared_local
-  moe_config lc = c;
-  lc.n_routed = expert_end - expert_begin;
-  lc.shared_inter = shared_local;
+  const DispatchPlace place{&c, T, idx, x, at<int32_t>(ws, L.chunk_hist),
+                            at<int32_t>(ws, L.pos_local), pos, src, x_perm};
   const int32_t* off_local = offsets + expert_begin;
   void* sbuf = shared_local > 0 ? at<void>(ws, L.s) : nullptr;
   st = run_experts(lc, T, x_perm, src, off_local, w1, w3, w2, x, ws1, ws3, ws2,
                    at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
-                   at<void>(ws, L.row_maps), err, s);
+                   at<void>(ws, L.row_maps), err, s, &place);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine_partial(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf,
                                             off_local, lc.n_routed, y_partial, s));
@@ -573,7 +595,7 @@ const char* moe_status_string(moe_status st) {
 int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
   if (check_config(cfg, T) != MOE_OK) return -1;
   // router: logits + select; dispatch: rank + scan + positions; experts: up
-  // + down, after one kernel that writes the per-expert A maps when the
+  // + down, with one kernel that writes the per-expert A maps when the
   // one-CTA tensor-core kernel runs; combine
   const bool row_maps = cfg->dtype == MOE_DT_BF16 && (g_expert_kernel == MOE_EXPERT_KERNEL_AUTO ||
                                                       g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05);
