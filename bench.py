@@ -459,9 +459,9 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     max over ranks; the timed loop records no other event. The per-kernel
     times come from a separate, untimed pass right after it (a tenth of the
     steps, 2 to 20), whose forwards record an event between every two kernels
-    and so run all their kernels on the one stream (the shared expert's
-    up-projection inside the routed experts' launch). Returns (ms, kernels_ms
-    per launch, kernels_ms_steps, clocks)."""
+    (and launch the up-projection as an ordinary launch, so each interval
+    holds one kernel). Returns (ms, kernels_ms per launch, kernels_ms_steps,
+    clocks)."""
     M = S.M
     clocks = Clocks() if clocks_on else None
     for _ in range(warmup):
@@ -489,8 +489,8 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     if M.moe_check_error(S.ws, S.stream) != M.MOE_OK:
         raise RuntimeError(f"{S.cfg.name}: device error word set during the timed loop")
     ck = clocks.stop(wall0, wall1, uuid) if clocks else None
-    rec = {"recorded": n_rec, "pass": "separate, untimed, after the timed loop; each recorded "
-                                      "forward runs its kernels on one stream"}
+    rec = {"recorded": n_rec, "pass": "separate, untimed, after the timed loop; a recorded "
+                                      "forward launches each kernel only after the one before"}
     return ms, {k: v / max(n_rec, 1) for k, v in stage_ms.items()}, rec, ck
 
 

@@ -215,8 +215,6 @@ struct GroupedArgs {
 void stage_mark(cudaStream_t st);
 // Whether the stage timer is recording the current forward call.
 bool stage_timing_active();
-// SMs of the current device (cached per device).
-int num_sms_current();
 
 // Router: logits (tensor cores for bf16 unless `simt`, else CUDA cores) into
 // `part` with at most `splits` k splits, then selection into weights / idx.
@@ -260,7 +258,7 @@ struct DispatchPlace {
   int32_t* src;
   void* x_perm;
 };
-cudaError_t launch_dispatch_place(const DispatchPlace& p, int num_sms, cudaStream_t st);
+cudaError_t launch_dispatch_place(const DispatchPlace& p, cudaStream_t st);
 cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, const int32_t* pos,
                            const float* weights, const void* s, void* y, cudaStream_t st);
 // Expert parallelism: one rank's fp32 share of y (pairs routed to its

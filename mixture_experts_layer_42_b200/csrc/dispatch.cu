@@ -163,45 +163,38 @@ dispatch_pos_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__
   if (p >= 0) src[p] = (int32_t)t;
 }
 
-// Persistent: a grid of a few CTAs per SM walks the (token, 4 KB slice)
-// items, so that every CTA is running from the start and a programmatic
-// dependent launch (the up-projection, whose shared-expert tiles need none
-// of this kernel's output) can start at once and overlap the copy.
+// Grid (token, 4 KB slice of the row). Lets a programmatic dependent launch
+// (the up-projection) start as soon as its last wave is running.
 template <typename T>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ pos_local,
-                        const int32_t* __restrict__ chunk_base, int64_t T_tok, int k, int E, int D,
+                        const int32_t* __restrict__ chunk_base, int k, int E, int D,
                         const T* __restrict__ x, int32_t* __restrict__ pos,
                         int32_t* __restrict__ src, T* __restrict__ x_perm) {
   asm volatile("griddepcontrol.launch_dependents;");
   __shared__ int32_t dst[32];
+  const int64_t t = blockIdx.x;
+  const int64_t chunk = t / kDispatchChunkTokens;
+  if (threadIdx.x < k) {
+    const int64_t q = t * k + threadIdx.x;
+    const int pl = pos_local[q];
+    int p = -1;
+    if (pl >= 0) p = chunk_base[chunk * E + idx[q]] + pl;
+    dst[threadIdx.x] = p;
+    if (blockIdx.y == 0) {
+      pos[q] = p;
+      if (p >= 0) src[p] = (int32_t)t;
+    }
+  }
+  __syncthreads();
   constexpr int VE = 16 / sizeof(T);
   const int nvec = D / VE;
-  const int nslice = (nvec + 255) / 256;
-  for (int64_t w = blockIdx.x; w < T_tok * nslice; w += gridDim.x) {
-    const int64_t t = w / nslice;
-    const int slice = (int)(w % nslice);
-    __syncthreads();  // the previous item's reads of dst are done
-    if (threadIdx.x < k) {
-      const int64_t q = t * k + threadIdx.x;
-      const int pl = pos_local[q];
-      int p = -1;
-      if (pl >= 0) p = chunk_base[(t / kDispatchChunkTokens) * E + idx[q]] + pl;
-      dst[threadIdx.x] = p;
-      if (slice == 0) {
-        pos[q] = p;
-        if (p >= 0) src[p] = (int32_t)t;
-      }
-    }
-    __syncthreads();
-    const int v = slice * 256 + threadIdx.x;
-    if (v < nvec) {
-      const uint4 val = reinterpret_cast<const uint4*>(x + t * D)[v];
-      for (int j = 0; j < k; ++j) {
-        const int p = dst[j];
-        if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * D)[v] = val;
-      }
-    }
+  const int v = blockIdx.y * blockDim.x + threadIdx.x;
+  if (v >= nvec) return;
+  const uint4 val = reinterpret_cast<const uint4*>(x + t * D)[v];
+  for (int j = 0; j < k; ++j) {
+    const int p = dst[j];
+    if (p >= 0) reinterpret_cast<uint4*>(x_perm + (int64_t)p * D)[v] = val;
   }
 }
 
@@ -223,7 +216,7 @@ cudaError_t launch_dispatch_sort(const moe_config& c, int64_t T, const int32_t* 
   return cudaSuccess;
 }
 
-cudaError_t launch_dispatch_place(const DispatchPlace& p, int num_sms, cudaStream_t st) {
+cudaError_t launch_dispatch_place(const DispatchPlace& p, cudaStream_t st) {
   const moe_config& c = *p.c;
   const int E = c.n_routed, k = c.topk, D = c.dim;
   if (p.x_perm == nullptr) {
@@ -235,19 +228,14 @@ cudaError_t launch_dispatch_place(const DispatchPlace& p, int num_sms, cudaStrea
   }
   const int ab = act_bytes(c);
   const int nvec = D * ab / 16;
-  const int64_t items = p.T * ceil_div(nvec, 256);
-  // 5 CTAs of 256 threads (26 registers each) per SM leave room beside them
-  // for one CTA of the expert GEMM (192 threads, 108 registers, 200 KB of
-  // shared memory), which may start on its shared-expert tiles meanwhile
-  const int64_t cap = (int64_t)(num_sms > 0 ? num_sms : 148) * 5;
-  const unsigned grid = (unsigned)(items < cap ? items : cap);
+  dim3 grid((unsigned)p.T, (unsigned)ceil_div(nvec, 256));
   if (c.dtype == MOE_DT_BF16)
     dispatch_scatter_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        p.idx, p.pos_local, p.chunk_hist, p.T, k, E, D, (const __nv_bfloat16*)p.x, p.pos, p.src,
+        p.idx, p.pos_local, p.chunk_hist, k, E, D, (const __nv_bfloat16*)p.x, p.pos, p.src,
         (__nv_bfloat16*)p.x_perm);
   else
-    dispatch_scatter_kernel<float><<<grid, 256, 0, st>>>(p.idx, p.pos_local, p.chunk_hist, p.T, k,
-                                                         E, D, (const float*)p.x, p.pos, p.src,
+    dispatch_scatter_kernel<float><<<grid, 256, 0, st>>>(p.idx, p.pos_local, p.chunk_hist, k, E, D,
+                                                         (const float*)p.x, p.pos, p.src,
                                                          (float*)p.x_perm);
   stage_mark(st);
   return cudaGetLastError();
@@ -261,7 +249,7 @@ cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, 
       launch_dispatch_sort(c, T, idx, counts, offsets, chunk_hist, pos_local, n_chunks, err, st);
   if (e != cudaSuccess) return e;
   DispatchPlace p{&c, T, idx, x, chunk_hist, pos_local, pos, src, x_perm};
-  return launch_dispatch_place(p, num_sms_current(), st);
+  return launch_dispatch_place(p, st);
 }
 
 }  // namespace moe

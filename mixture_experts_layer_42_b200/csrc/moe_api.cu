@@ -51,8 +51,6 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(ws) + off);
 }
 
-}  // namespace
-
 int num_sms_current() {
   static int cached[64] = {0};
   int dev = 0;
@@ -66,8 +64,6 @@ int num_sms_current() {
   }
   return cached[dev];
 }
-
-namespace {
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -130,7 +126,7 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
       e = launch_row_maps(h, Tk, c.moe_inter, x_perm, c.dim, offsets, c.n_routed, row_maps, ctr, st);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     }
-    if (place != nullptr && launch_dispatch_place(*place, num_sms_current(), st) != cudaSuccess)
+    if (place != nullptr && launch_dispatch_place(*place, st) != cudaSuccess)
       return MOE_ERR_CUDA;
     // (not while the stage timer records events between the launches)
     const bool pdl = place != nullptr && kind == TC_ROWS && !stage_timing_active();
@@ -145,7 +141,7 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
                           num_sms_current(), st, false);
     return cuda_status(e);
   }
-  if (place != nullptr && launch_dispatch_place(*place, num_sms_current(), st) != cudaSuccess)
+  if (place != nullptr && launch_dispatch_place(*place, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   GroupedArgs g;
   memset(&g, 0, sizeof(g));
