@@ -1,23 +1,28 @@
 // Grouped SwiGLU expert GEMMs with FP8 (e4m3) block-scaled weights and
-// activations, on the 5th-generation tensor cores (tcgen05.mma kind::f8f6f4).
+// activations, on the 5th-generation tensor cores (tcgen05.mma
+// kind::mxf8f6f4 with block scaling: the tensor core applies the scales).
 //
 // The pages say only that the block's other linears are FP8 ("Expert
 // scores", dtype note). The layout here is this library's: e4m3 values, one
 // power-of-two fp32 scale per 128 x 128 block of a weight matrix [out, in]
 // and per 1 x 128 block of a row of activations (the smallest scale that
-// keeps the block within 448). x is quantized once per step (quant_rows
+// keeps the block within 448, and at least 2^-127, so that every scale is one
+// UE8M0 byte). x is quantized once per step (quant_rows
 // kernel); h = silu(w1 x) * (w3 x) is quantized by the up-projection's
 // epilogue; each expert's output is bf16, as on the bf16 path.
 //
 // Tiles put the weights on the MMA's M side (128 rows: one scale block) and
-// up to NT tokens of one expert on its N side (rounded up to 16), so a decode
-// batch (a few tokens per expert) does little MMA work while it streams the
-// active experts' weights at half the bytes of bf16. Each 128-deep k-block
-// (one scale block) is accumulated by the tensor core into a fresh fp32 TMEM
-// buffer, and the four epilogue warps add it into register sums with the
-// product of its weight scale and each token's activation scale:
-//   sum[f, t] += s_w(e, f/128, kb) * s_x(t, kb) * sum_{k in kb} q_w[f, k] q_x[t, k]
-// (a lane of TMEM is a weight row f, a column a token t).
+// up to NT = 32 tokens of one expert on its N side, so a decode batch (a few
+// tokens per expert) does little MMA work while it streams the active
+// experts' weights at half the bytes of bf16. Every MMA is block-scaled: per
+// 32-deep slice of K it multiplies each weight row by its UE8M0 scale and each
+// token by its own, so one fp32 TMEM accumulator sums the whole K,
+//   sum[f, t] = sum_kb s_w(e, f/128, kb) s_x(t, kb) sum_{k in kb} q_w[f, k] q_x[t, k]
+// (a lane of TMEM is a weight row f, a column a token t), and the epilogue
+// reads it once per tile. The producer writes each stage's scale bytes to
+// shared memory (the weight block's byte in all 128 rows, each token's byte
+// in its row) and the MMA thread copies them to TMEM (tcgen05.cp
+// 32x128b.warpx4) before that stage's MMAs.
 //
 // One CTA per SM, 192 threads: warp 0 TMA (weights by tile, token rows by
 // tile::gather4 from the routed rows' tokens or the rows themselves; rows
@@ -47,37 +52,72 @@ constexpr int MAX_STAGES = 9;
 constexpr int RING_BYTES = 9 * (A_BYTES + W_BYTES);  // the larger of the two rings (184 KB)
 static_assert(5 * (A_BYTES + 2 * W_BYTES) <= RING_BYTES, "UP ring");
 constexpr int NTHREADS = 192;
-constexpr uint32_t FTMEM = 512;
+constexpr uint32_t FTMEM = 256;
 constexpr int MAXE = 1024;
 constexpr int MAX_KB = 64;                     // k-blocks per tile (K <= 8192)
-constexpr int NBUF_UP = 8;                     // TMEM buffers of 2 x NT columns
-constexpr int NBUF_DOWN = 16;                  // TMEM buffers of NT columns
-// The epilogue drains k-blocks KG at a time: one barrier wait (on the
-// group's last buffer: commits complete in order) and one tcgen05.wait::ld
-// per group instead of per k-block, so their latencies do not pace the
-// pipeline (one k-block at a time, the FP8 up-projection of a 32-expert
-// decode batch took longer than the bf16 one for half the bytes).
-constexpr int KG = 4;
-constexpr int SC_SLOT = NT * MAX_KB * 4;      // one tile's token scales (16 KB)
-// alignment slack, stages, barriers (512), P and off, 16 bytes to align the
-// scale slots, the two scale slots, the per-warp maxima
-constexpr size_t FSMEM = 1024 + (size_t)RING_BYTES + 512 + 2 * (MAXE + 1) * 4 + 16 +
-                         2 * (size_t)SC_SLOT + 4 * NT * 4;
+// TMEM columns: two accumulator buffers (the epilogue drains one tile while
+// the next accumulates), each 2 x NT columns for UP (w1 rows | w3 rows) and
+// NT for DOWN, from column 0; then per stage the scale factors the MMAs of
+// that stage read: 4 columns for the weight rows' (SFA; w1 and w3 each for
+// UP) and 4 for the tokens' (SFB; only the first is read at N = 32).
+constexpr int ACC_COLS_UP = 2 * NT, ACC_COLS_DOWN = NT;
+constexpr int SF_COL0 = 2 * ACC_COLS_UP;
+template <bool UP> struct SfCols {
+  static constexpr int PER_STAGE = UP ? 12 : 8;
+};
+static_assert(SF_COL0 + 5 * 12 <= (int)FTMEM && SF_COL0 + 9 * 8 <= (int)FTMEM, "TMEM columns");
+// Per stage in shared memory, the scale-factor bytes the MMA thread copies to
+// TMEM (tcgen05.cp 32x128b.warpx4): 512 bytes each for SFA (w1), SFA (w3, UP)
+// and SFB, row r = TMEM lane r of each of the four sub-partitions.
+constexpr int SF_BYTES = 512;
+constexpr int SF_STAGE_MAX = 3 * SF_BYTES;
+constexpr int SC_SLOT = NT * MAX_KB * 4;      // one tile's token scales (8 KB)
+// alignment slack, stages, the stages' scale-factor bytes, barriers (512), P
+// and off, 16 bytes to align the scale slots, the two scale slots, the
+// per-warp maxima
+constexpr size_t FSMEM = 1024 + (size_t)RING_BYTES + 9 * 2 * SF_BYTES + 512 +
+                         2 * (MAXE + 1) * 4 + 16 + 2 * (size_t)SC_SLOT + 4 * NT * 4;
+static_assert(5 * 3 * SF_BYTES <= 9 * 2 * SF_BYTES, "UP scale-factor bytes");
 
-// kind::f8f6f4 instruction descriptor: fp32 accumulator, e4m3 A and B, both
-// K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// kind::mxf8f6f4 block-scaled instruction descriptor: e4m3 A and B, both
+// K-major, fp32 accumulator, UE8M0 scale factors (bit 23), scale-factor byte
+// 0 of A's and B's TMEM words (bits 29-30, 4-5), M x N.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N) {
+  return ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
+// D[M x N] (+)= (A * 2^SFA) (B * 2^SFB)^T over K = 32: one UE8M0 scale per row
+// of A and per row of B (tcgen05 block scaling, one scale vector per 32 K).
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                       uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
       : "memory");
+}
+
+// Shared-memory descriptor of a 32 x 16-byte matrix, no swizzle, rows 16
+// bytes apart (8-row core matrices 128 bytes apart): the source of a
+// tcgen05.cp 32x128b.
+__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)(128 >> 4) << 16) |
+         ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
+}
+
+// TMEM lanes 32w + r (w = 0..3) <- shared row r (16 bytes), r = 0..31.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// The UE8M0 byte of a power-of-two scale 2^s, -127 <= s <= 127: the biased
+// exponent field of its fp32 encoding (2^-127 is the subnormal with a zero
+// exponent field, which is UE8M0's code 0).
+__device__ __forceinline__ uint32_t ue8m0(float scale) {
+  return (__float_as_uint(scale) >> 23) & 0xFFu;
 }
 
 struct Fp8Args {
@@ -85,9 +125,9 @@ struct Fp8Args {
   // (UP: the quantized x, read by token through src; DOWN: the quantized h
   // in expert order), [1] the shared MLP's (UP: quantized x; DOWN: its h)
   CUtensorMap tmA[2];
-  // the same tensors for tile loads of contiguous rows (boxes of 16 and 32
-  // rows): every A but the routed UP's, whose rows are gathered by token
-  CUtensorMap tmAt[2][2];
+  // the same tensors for tile loads of NT contiguous rows: every A but the
+  // routed UP's, whose rows are gathered by token
+  CUtensorMap tmAt[2];
   CUtensorMap tmW1[2];   // weights [E, N, K] uint8, box 128 x 128 x 1: w1 (UP) / w2 (DOWN); shared E = 1
   CUtensorMap tmW3[2];   // w3 / ws3 (UP)
   const float* ws1[2];   // weight scales [E, N/128, K/128] of tmW1
@@ -155,13 +195,16 @@ __device__ __forceinline__ int round16(int r) { return (r + 15) & ~15; }
 // tile's rows can be copied in one bulk copy.
 __host__ __device__ __forceinline__ int scale_stride(int K) { return ((K / QB) + 3) & ~3; }
 
-// Smallest s with amax <= 448 * 2^s (0 for amax == 0): amax = m 2^e with
-// 0.5 <= m < 1, so s = e - 9, plus one when 2m > 1.75.
+// Smallest s with amax <= 448 * 2^s (0 for amax == 0), and at least -127,
+// the smallest scale UE8M0 encodes (blocks whose largest magnitude is below
+// 448 * 2^-127 keep that scale): amax = m 2^e with 0.5 <= m < 1, so s = e - 9,
+// plus one when 2m > 1.75.
 __device__ __forceinline__ int block_exp(float amax) {
   if (!(amax > 0.f)) return 0;
   int e;
   const float m = frexpf(amax, &e);
-  return e - 9 + (2.f * m > 1.75f ? 1 : 0);
+  const int s = e - 9 + (2.f * m > 1.75f ? 1 : 0);
+  return s < -127 ? -127 : s;
 }
 
 // (Values are brought into range with ldexpf(v, -s): the reciprocal 2^-s of
@@ -192,23 +235,23 @@ template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  constexpr int NBUF = UP ? NBUF_UP : NBUF_DOWN;
-  constexpr int BUF_COLS = UP ? 2 * NT : NT;
+  constexpr int ACC_COLS = UP ? ACC_COLS_UP : ACC_COLS_DOWN;
   constexpr int FSTAGES = Ring<UP>::STAGES;
   constexpr int FSTAGE = Ring<UP>::BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + RING_BYTES);
+  constexpr int SF_STAGE = (UP ? 3 : 2) * SF_BYTES;   // SFA (w1), [SFA (w3)], SFB
+  uint8_t* sfs = tiles + RING_BYTES;                  // [FSTAGES][SF_STAGE]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sfs + 9 * 2 * SF_BYTES);
   uint64_t* empty = full + FSTAGES;
   uint64_t* tfull = empty + FSTAGES;
-  uint64_t* tempty = tfull + NBUF;
-  uint64_t* drain = tempty + NBUF;
-  uint64_t* sfull = drain + 1;            // token-scale slots: copied in
-  uint64_t* sempty = sfull + 2;           //                    read by the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + 2);
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint64_t* sfull = drain + 1;            // token-scale slots, copied in by the producer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfull + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* P = reinterpret_cast<int32_t*>(tiles + RING_BYTES + 512);
+  int32_t* P = reinterpret_cast<int32_t*>(sfs + 9 * 2 * SF_BYTES + 512);
   int32_t* off = P + MAXE + 1;
   // [2][rows][K/128] the token scales of a tile (two slots, copied in bulk
-  // by the producer a tile ahead), then [4][NT] per-warp maxima
+  // a tile ahead), then [4][NT] per-warp maxima
   float* tsc = reinterpret_cast<float*>(off + MAXE + 1 + 2);  // 16-byte aligned
   float* red = tsc + 2 * NT * MAX_KB;
 
@@ -218,8 +261,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
   if (warp == 0) {
     if (lane == 0) {
       for (int s = 0; s < FSTAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-      for (int b = 0; b < NBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
-      for (int b = 0; b < 2; ++b) { mbar_init(&sfull[b], 1); mbar_init(&sempty[b], 128); }
+      for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+      for (int b = 0; b < 2; ++b) mbar_init(&sfull[b], 1);
       mbar_init(drain, 1);
       *abort_flag = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -277,37 +320,62 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // lane 0: barriers and the weight tiles; lanes 0..n16/4-1: 4 token rows
-    // each by tile::gather4
+    // Lane 0: barriers, the weight tiles and a contiguous tile's token rows;
+    // lanes 0..NT/4-1 gather 4 token rows each (routed UP). Every lane writes
+    // its row of each stage's scale-factor bytes: the weight block's scale
+    // (the same for all 128 weight rows of the tile) and its token's.
     int s = 0, issued = 0, scopies = 0;
     uint32_t ph = 0;
     bool ok = true;
+    if (lane == 0 && (int)blockIdx.x < S.total) {   // the first tile's token scales
+      const Tile t0 = decode(S, blockIdx.x);
+      const int kbp = scale_stride(g.kdim[t0.kind]);
+      const uint32_t bytes = (uint32_t)(t0.rows * kbp * 4);
+      mbar_expect_tx(&sfull[0], bytes);
+      bulk_load(tsc, g.asc[t0.kind] + (int64_t)t0.row0 * kbp, bytes, &sfull[0]);
+      ++scopies;
+    }
     for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
       const Tile t = decode(S, i);
       const int kb_n = g.kdim[t.kind] / QB;
-      const int n16 = round16(t.rows);
-      // the tile's token scales: t.rows contiguous rows of kb_n floats
+      const int kbp = scale_stride(g.kdim[t.kind]);
+      const int slot = lt & 1;
+      // the tile's weight scales as UE8M0 bytes, k-blocks lane and lane + 32
+      const int nbw = g.n_out[t.kind] / QB;
+      const float* pw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
+      const uint32_t w1a = lane < kb_n ? ue8m0(__ldg(pw1 + lane)) : 127u;
+      const uint32_t w1b = lane + 32 < kb_n ? ue8m0(__ldg(pw1 + lane + 32)) : 127u;
+      uint32_t w3a = 127u, w3b = 127u;
+      if (UP) {
+        const float* pw3 = g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
+        w3a = lane < kb_n ? ue8m0(__ldg(pw3 + lane)) : 127u;
+        w3b = lane + 32 < kb_n ? ue8m0(__ldg(pw3 + lane + 32)) : 127u;
+      }
+      // this tile's token scales (copied a tile ahead), then the next tile's
+      // copy into the other slot (its last reader, the previous tile's loop
+      // below, is done: the warp has synchronised since)
       {
         int w = 1;
-        if (lane == 0) {
-          const int slot = lt & 1;
-          w = mbar_wait(&sempty[slot], ((lt >> 1) & 1) ^ 1, abort_flag, g.err) ? 1 : 0;
-          if (w) {
-            const int kbp = scale_stride(g.kdim[t.kind]);
-            const uint32_t bytes = (uint32_t)(t.rows * kbp * 4);
-            mbar_expect_tx(&sfull[slot], bytes);
-            bulk_load(tsc + slot * NT * MAX_KB, g.asc[t.kind] + (int64_t)t.row0 * kbp, bytes,
-                      &sfull[slot]);
-            ++scopies;
-          }
-        }
+        if (lane == 0) w = mbar_wait(&sfull[slot], (uint32_t)(lt >> 1) & 1, abort_flag, g.err) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
       }
-      const int n_g = n16 / 4;
+      if (lane == 0 && i + (int)gridDim.x < S.total) {
+        const Tile tn = decode(S, i + gridDim.x);
+        const int kbpn = scale_stride(g.kdim[tn.kind]);
+        const uint32_t bytes = (uint32_t)(tn.rows * kbpn * 4);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(&sfull[slot ^ 1], bytes);
+        bulk_load(tsc + (slot ^ 1) * NT * MAX_KB, g.asc[tn.kind] + (int64_t)tn.row0 * kbpn, bytes,
+                  &sfull[slot ^ 1]);
+        ++scopies;
+      }
+      const float* ts = tsc + slot * NT * MAX_KB;   // [t.rows][kbp]
       // routed UP rows are tokens scattered over x: gathered four at a time;
-      // the others (expert-ordered h, token rows) are contiguous: one tile load
+      // the others (expert-ordered h, token rows) are contiguous: one tile
+      // load of NT rows (rows past a tile's tokens are multiplied and not
+      // stored; past the tensor's end they read zeros)
       const bool gath = UP && t.kind == 0;
-      const uint32_t tx = (uint32_t)(n16 * QB + (UP ? 2 : 1) * W_BYTES);
+      const uint32_t tx = (uint32_t)(NT * QB + (UP ? 2 : 1) * W_BYTES);
       int r[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -321,17 +389,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        // the stage's scale factors (the stage's previous MMAs, and the copies
+        // to TMEM before them, are complete: empty[s] came from their commit)
+        uint8_t* sf = sfs + s * SF_STAGE;
+        const uint32_t b1 = __shfl_sync(0xffffffffu, kb < 32 ? w1a : w1b, kb & 31) * 0x01010101u;
+        *reinterpret_cast<uint4*>(sf + lane * 16) = make_uint4(b1, b1, b1, b1);
+        if (UP) {
+          const uint32_t b3 = __shfl_sync(0xffffffffu, kb < 32 ? w3a : w3b, kb & 31) * 0x01010101u;
+          *reinterpret_cast<uint4*>(sf + SF_BYTES + lane * 16) = make_uint4(b3, b3, b3, b3);
+        }
+        const uint32_t bt = (lane < t.rows ? ue8m0(ts[lane * kbp + kb]) : 127u) * 0x01010101u;
+        *reinterpret_cast<uint4*>(sf + (UP ? 2 : 1) * SF_BYTES + lane * 16) = make_uint4(bt, bt, bt, bt);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
         uint8_t* sa = tiles + s * FSTAGE;
         uint8_t* sw = sa + A_BYTES;
         if (lane == 0) {
           mbar_expect_tx(&full[s], tx);
           tma_load_3d(sw, &g.tmW1[t.kind], &full[s], kb * QB, t.n0, t.e);
           if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], kb * QB, t.n0, t.e);
+          if (!gath) tma_load_2d(sa, &g.tmAt[t.kind], &full[s], kb * QB, t.row0);
         }
-        if (!gath && lane == 0)   // contiguous rows: one tile load (rows past the end read zeros)
-          tma_load_2d(sa, &g.tmAt[t.kind][n16 > 16 ? 1 : 0], &full[s], kb * QB, t.row0);
         __syncwarp();
-        if (gath && lane < n_g)
+        if (gath && lane < NT / 4)
           tma_gather4(sa + lane * (4 * QB), &g.tmA[t.kind], &full[s], kb * QB, r[0], r[1], r[2], r[3]);
         ++issued;
         if (++s == FSTAGES) { s = 0; ph ^= 1; }
@@ -350,116 +430,87 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // Per stage: the scale factors to TMEM (tcgen05.cp, ordered before the
+    // MMAs this thread issues after it), then four K = 32 block-scaled MMAs
+    // (eight for UP: w1 and w3) into the tile's accumulator, which sums the
+    // whole K; one commit per tile hands it to the epilogue.
     if (lane == 0) {
-      int s = 0, u = 0;  // u: k-blocks issued so far (TMEM buffer rotation)
+      int s = 0;
       uint32_t ph = 0;
       bool ok = true;
-      for (int i = blockIdx.x; ok && i < S.total; i += gridDim.x) {
+      const uint32_t idesc = idesc_mx_e4m3(QB, NT);
+      for (int i = blockIdx.x, lt = 0; ok && i < S.total; i += gridDim.x, ++lt) {
         const Tile t = decode(S, i);
         const int kb_n = g.kdim[t.kind] / QB;
-        const uint32_t idesc = idesc_e4m3(QB, round16(t.rows));
-        for (int kb = 0; kb < kb_n; ++kb, ++u) {
-          const int b = u % NBUF;
-          const uint32_t use = (uint32_t)(u / NBUF);
-          if (!mbar_wait(&tempty[b], (use & 1) ^ 1, abort_flag, g.err)) { ok = false; break; }
-          tc_fence_after();
+        const int b = lt & 1;
+        if (!mbar_wait(&tempty[b], ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag, g.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(b * ACC_COLS);
+        for (int kb = 0; kb < kb_n; ++kb) {
           if (!mbar_wait(&full[s], ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(tiles + s * FSTAGE);
           const uint32_t w0 = a0 + A_BYTES;
-          const uint32_t d = tmem_base + (uint32_t)(b * BUF_COLS);
+          const uint32_t sf0 = smem_u32(sfs + s * SF_STAGE);
+          const uint32_t tsa = tmem_base + (uint32_t)(SF_COL0 + s * SfCols<UP>::PER_STAGE);
+          const uint32_t tsb = tsa + (UP ? 8 : 4);
+          tmem_cp_sf(tsa, sdesc_sf(sf0));
+          if (UP) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
+          tmem_cp_sf(tsb, sdesc_sf(sf0 + (UP ? 2 : 1) * SF_BYTES));
 #pragma unroll
           for (int kk = 0; kk < QB / 32; ++kk) {
-            mma_f8(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, kk != 0 ? 1u : 0u);
-            if (UP) mma_f8(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc,
-                           kk != 0 ? 1u : 0u);
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            mma_mx(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, tsa, tsb, acc);
+            if (UP) mma_mx(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc, tsa + 4,
+                           tsb, acc);
           }
           tc_commit(&empty[s]);
-          tc_commit(&tfull[b]);
           if (++s == FSTAGES) { s = 0; ph ^= 1; }
         }
+        if (!ok) break;
+        tc_commit(&tfull[b]);
       }
       tc_commit(drain);
       mbar_drain(drain, 0);
     }
   } else {
     // ---------------------------------------------------------------- epilogue
+    // The tile's fp32 sums (scales already applied by the tensor core): a
+    // TMEM lane is a weight row f, a column a token.
     const int quad = warp & 3;
     const int f = quad * 32 + lane;      // this thread's weight row (TMEM lane) in the tile
     const int et = threadIdx.x - 64;     // 0..127 among the epilogue threads
-    int u = 0;
     for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
       const Tile t = decode(S, i);
-      const int kb_n = g.kdim[t.kind] / QB;
-      const int n16 = round16(t.rows);
-      bool ok = true;
-      // the tile's token scales, copied in by the producer
-      const int slot = lt & 1;
+      const int b = lt & 1;
+      bool ok;
       {
         int w = 1;
-        if (lane == 0) w = mbar_wait(&sfull[slot], (lt >> 1) & 1, abort_flag, g.err) ? 1 : 0;
+        if (lane == 0) w = mbar_wait(&tfull[b], (uint32_t)(lt >> 1) & 1, abort_flag, g.err) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       }
-      const float* sc = tsc + slot * NT * MAX_KB;   // [t.rows][kbp]
-      const int kbp = scale_stride(g.kdim[t.kind]);
-      const int nbw = g.n_out[t.kind] / QB;
-      const float* sw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
-      const float* sw3 = UP ? g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n : nullptr;
       float sa[NT], sb[UP ? NT : 1];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) { sa[j] = 0.f; if (UP) sb[j] = 0.f; }
-      for (int kb = 0; ok && kb < kb_n; kb += KG) {
-        const int gc = kb_n - kb < KG ? kb_n - kb : KG;   // k-blocks in this group
-        {
-          const int ul = u + gc - 1;
-          int w = 1;
-          if (lane == 0) w = mbar_wait(&tfull[ul % NBUF], (uint32_t)(ul / NBUF) & 1, abort_flag, g.err) ? 1 : 0;
-          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        }
+      if (ok) {
         tc_fence_after();
-        float c1[KG], c3[KG];
+        const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * ACC_COLS);
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tb, r0);
+        tmem_ld16(tb + 16, r1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < KG; ++q) {
-          c1[q] = q < gc ? __ldg(sw1 + kb + q) : 0.f;
-          c3[q] = (UP && q < gc) ? __ldg(sw3 + kb + q) : 0.f;
-        }
+        for (int j = 0; j < 16; ++j) { sa[j] = __uint_as_float(r0[j]); sa[16 + j] = __uint_as_float(r1[j]); }
+        if (UP) {
+          tmem_ld16(tb + NT, r0);
+          tmem_ld16(tb + NT + 16, r1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j0 = 0; j0 < NT; j0 += 16) {
-          if (j0 < n16) {
-            uint32_t ra[KG][16], rb[KG][UP ? 16 : 1];
-#pragma unroll
-            for (int q = 0; q < KG; ++q) {
-              if (q < gc) {
-                const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) +
-                                    (uint32_t)(((u + q) % NBUF) * BUF_COLS);
-                tmem_ld16(tb + j0, ra[q]);
-                if (UP) tmem_ld16(tb + NT + j0, *reinterpret_cast<uint32_t(*)[16]>(rb[q]));
-              }
-            }
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < KG; ++q) {
-              if (q < gc) {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                  // rows past the tile's tokens: their products are zero, and
-                  // the slot holds no scale for them
-                  const float xs = (j0 + c < t.rows) ? sc[(j0 + c) * kbp + kb + q] : 0.f;
-                  sa[j0 + c] = fmaf(__uint_as_float(ra[q][c]), c1[q] * xs, sa[j0 + c]);
-                  if (UP) sb[j0 + c] = fmaf(__uint_as_float(rb[q][c]), c3[q] * xs, sb[j0 + c]);
-                }
-              }
-            }
-          }
+          for (int j = 0; j < 16; ++j) { sb[j] = __uint_as_float(r0[j]); sb[16 + j] = __uint_as_float(r1[j]); }
         }
         tc_fence_before();
-        for (int q = 0; q < gc; ++q) mbar_arrive(&tempty[(u + q) % NBUF]);
-        u += gc;
+        mbar_arrive(&tempty[b]);
       }
-      // one decision for all four warps: stop if any of them gave up; the
-      // scale slot is free once every epilogue thread is past its last read
+      // one decision for all four warps: stop if any of them gave up
       if (epi_sync_any(!ok)) break;
-      mbar_arrive(&sempty[slot]);
       if (UP) {
         // h = silu(a) * b, quantized per token over this tile's 128 features
         // (one 1 x 128 block of h's row)
@@ -468,7 +519,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         const int nbh = scale_stride(g.n_out[t.kind]);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          if (j >= n16) break;
           const float h = silu_f(sa[j]) * sb[j];
           sa[j] = h;
           float m = fabsf(h);
@@ -705,20 +755,17 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
         g.out[1] = s;
       }
     }
-    // tile-load maps of the A tensors (boxes of 16 and 32 rows)
+    // tile-load maps of the A tensors (boxes of NT rows)
     {
       const void* a0p = up ? (const void*)xq : (const void*)hq;
       const uint64_t r0 = up ? (uint64_t)T : (uint64_t)Tk, kk0 = up ? (uint64_t)D : (uint64_t)I;
-      for (int b = 0; b < 2; ++b)
-        if (!map_u8_tile(&g.tmAt[0][b], a0p, r0, kk0, 16u << b)) return cudaErrorInvalidValue;
+      if (!map_u8_tile(&g.tmAt[0], a0p, r0, kk0, NT)) return cudaErrorInvalidValue;
       if (sh) {
         const void* a1p = up ? (const void*)xq : (const void*)hsq;
         const uint64_t kk1 = up ? (uint64_t)D : (uint64_t)Is;
-        for (int b = 0; b < 2; ++b)
-          if (!map_u8_tile(&g.tmAt[1][b], a1p, (uint64_t)T, kk1, 16u << b)) return cudaErrorInvalidValue;
+        if (!map_u8_tile(&g.tmAt[1], a1p, (uint64_t)T, kk1, NT)) return cudaErrorInvalidValue;
       } else {
-        g.tmAt[1][0] = g.tmAt[0][0];
-        g.tmAt[1][1] = g.tmAt[0][1];
+        g.tmAt[1] = g.tmAt[0];
       }
     }
     if (!sh) {  // no shared group: its maps are never used, keep them valid

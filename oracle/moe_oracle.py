@@ -107,12 +107,18 @@ def round_e4m3(v: np.ndarray) -> np.ndarray:
     return np.clip(out, -E4M3_MAX, E4M3_MAX)
 
 
+SCALE_EXP_MIN = -127   # the smallest power of two a UE8M0 scale byte encodes
+
+
 def block_exponent(amax: np.ndarray) -> np.ndarray:
-    """Smallest integer s with amax <= 448 * 2^s (0 for an all-zero block)."""
+    """Smallest integer s >= SCALE_EXP_MIN with amax <= 448 * 2^s (0 for an
+    all-zero block). The lower limit keeps every scale encodable as one UE8M0
+    byte (2^-127 .. 2^127), the form the tensor core's block scaling reads; a
+    block whose largest magnitude is below 448 * 2^-127 keeps 2^-127."""
     amax = np.asarray(amax, dtype=np.float64)
     m, e = np.frexp(np.where(amax > 0, amax, 1.0))   # amax = m 2^e, 0.5 <= m < 1
     # amax = (2m) 2^(e-1) and 448 = 1.75 * 2^8: s = e - 9, one more when 2m > 1.75
-    s = e - 9 + (2.0 * m > 1.75)
+    s = np.maximum(e - 9 + (2.0 * m > 1.75), SCALE_EXP_MIN)
     return np.where(amax > 0, s, 0).astype(np.int64)
 
 

@@ -55,6 +55,18 @@ def test_block_exponent_is_the_smallest_that_fits():
     assert O.block_exponent(np.array([0.0]))[0] == 0
 
 
+def test_block_exponent_stops_at_the_smallest_ue8m0_scale():
+    # 448 * 2^-127 is the largest magnitude the scale 2^-127 serves exactly;
+    # anything smaller keeps 2^-127 (a UE8M0 byte encodes 2^-127 .. 2^127)
+    edge = 448.0 * 2.0 ** -127
+    amax = np.array([edge, edge * (1 + 2 ** -20), edge / 2, 2.0 ** -120, 2.0 ** -140, 2.0 ** -1074])
+    np.testing.assert_array_equal(O.block_exponent(amax), [-127, -126, -127, -127, -127, -127])
+    # above the limit the rule is unchanged: 448 * 2^-126 needs exactly -126
+    assert O.block_exponent(np.array([448.0 * 2.0 ** -126]))[0] == -126
+    # the largest bf16 value needs 2^120, well inside the range
+    assert O.block_exponent(np.array([3.3895313892515355e38]))[0] == 120
+
+
 @pytest.mark.parametrize("br,bc,shape", [(128, 128, (300, 200)), (1, 128, (7, 300)), (128, 128, (128, 128))])
 def test_quantize_blocks_properties(br, bc, shape):
     rng = np.random.default_rng(2)
@@ -130,6 +142,7 @@ def pin_fp8():
     """The FP8 pins in one call (used by the planted-mistake tests)."""
     test_round_e4m3_known_values()
     test_block_exponent_is_the_smallest_that_fits()
+    test_block_exponent_stops_at_the_smallest_ue8m0_scale()
     for case in [(128, 128, (300, 200)), (1, 128, (7, 300))]:
         test_quantize_blocks_properties(*case)
     test_swiglu_fp8_matches_torch_restatement()

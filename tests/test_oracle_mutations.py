@@ -91,10 +91,11 @@ MUTATIONS = [
      "normal = np.ldexp(np.round(m * 32.0) / 32.0, e)", [TF8.pin_fp8]),
     ("e4m3 subnormal step 2^-8", "sub = np.round(v * 512.0) / 512.0", "sub = np.round(v * 256.0) / 256.0",
      [TF8.pin_fp8]),
-    ("fp8 scale one step too large", "s = e - 9 + (2.0 * m > 1.75)", "s = e - 8 + (2.0 * m > 1.75)",
+    ("fp8 scale one step too large", "s = np.maximum(e - 9 + (2.0 * m > 1.75)", "s = np.maximum(e - 8 + (2.0 * m > 1.75)",
      [TF8.pin_fp8]),
-    ("fp8 scale ignores the 1.75 boundary", "s = e - 9 + (2.0 * m > 1.75)", "s = e - 9 + (2.0 * m > 1.5)",
-     [TF8.pin_fp8]),
+    ("fp8 scale ignores the 1.75 boundary", "s = np.maximum(e - 9 + (2.0 * m > 1.75)",
+     "s = np.maximum(e - 9 + (2.0 * m > 1.5)", [TF8.pin_fp8]),
+    ("fp8 scale below the UE8M0 range", "SCALE_EXP_MIN = -127 ", "SCALE_EXP_MIN = -150 ", [TF8.pin_fp8]),
     ("h not quantized before w2", "h = fp8_act(silu(a) * c)", "h = silu(a) * c", [TF8.pin_fp8]),
     ("activations quantized per 128 x 128", "q, s = quantize_blocks(a, 1, 128)",
      "q, s = quantize_blocks(a, 128, 128)", [TF8.pin_fp8]),
