@@ -224,7 +224,9 @@ MOE_API moe_status moe_cast_output(const moe_config* cfg, int64_t T, const float
  * e4m3 values (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; finite
  * values up to 448), one fp32 scale per 128 x 128 block of each [out, in]
  * matrix, a power of two: the smallest 2^s with the block's largest magnitude
- * <= 448 * 2^s. A weight is q * scale. moe_quantize_fp8 produces the layout
+ * <= 448 * 2^s, and s >= -127 (so that every scale is one UE8M0 byte, the
+ * form the tensor core's block scaling reads; a block below 448 * 2^-127
+ * keeps 2^-127). A weight is q * scale. moe_quantize_fp8 produces the layout
  * from bf16 or fp32 weights. Scales are row-major over the blocks:
  * w1_scale / w3_scale [E, I/128, D/128], w2_scale [E, D/128, I/128],
  * ws1_scale / ws3_scale [I_s/128, D/128], ws2_scale [D/128, I_s/128]. */
@@ -261,9 +263,10 @@ MOE_API moe_status moe_workspace_size_fp8(const moe_config* cfg, int64_t T, size
 /* The whole layer with FP8 expert weights: the router as in moe_forward (bf16
  * W_r applied in fp32), then x quantized per 1 x 128 block of each row to
  * e4m3 (as the weights, one power-of-two scale per block), the routed and
- * shared SwiGLU experts on the e4m3 tensor cores (kind::f8f6f4, fp32
- * accumulation in 128-deep blocks scaled by the product of the weight's and
- * the row's block scales), h = silu(w1 x) * (w3 x) quantized the same way
+ * shared SwiGLU experts on the e4m3 tensor cores (kind::mxf8f6f4 block
+ * scaling: each product scaled by the weight's and the row's block scales
+ * inside the tensor core, one fp32 accumulation over K), h = silu(w1 x) *
+ * (w3 x) quantized the same way
  * before w2, each expert's output rounded to bf16, and the combine as in
  * moe_forward. Workspace of moe_workspace_size_fp8() bytes, initialised by
  * moe_workspace_init(). bf16 layers only. */
