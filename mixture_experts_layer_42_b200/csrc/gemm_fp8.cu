@@ -48,7 +48,6 @@ template <bool UP> struct Ring {
   static constexpr int STAGES = UP ? 5 : 9;
   static constexpr int BYTES = A_BYTES + (UP ? 2 : 1) * W_BYTES;
 };
-constexpr int MAX_STAGES = 9;
 constexpr int RING_BYTES = 9 * (A_BYTES + W_BYTES);  // the larger of the two rings (184 KB)
 static_assert(5 * (A_BYTES + 2 * W_BYTES) <= RING_BYTES, "UP ring");
 constexpr int NTHREADS = 192;
@@ -57,20 +56,27 @@ constexpr int MAXE = 1024;
 constexpr int MAX_KB = 64;                     // k-blocks per tile (K <= 8192)
 // TMEM columns: two accumulator buffers (the epilogue drains one tile while
 // the next accumulates), each 2 x NT columns for UP (w1 rows | w3 rows) and
-// NT for DOWN, from column 0; then per stage the scale factors the MMAs of
-// that stage read: 4 columns for the weight rows' (SFA; w1 and w3 each for
-// UP) and 4 for the tokens' (SFB; only the first is read at N = 32).
+// NT for DOWN, from column 0; then SF_SLOTS slots of scale factors, one per
+// group of up to four k-blocks of a tile: 4 columns for the weight rows'
+// (SFA; w1 and w3 each for UP) and 4 for the tokens' (SFB; only the first is
+// read at N = 32). Byte j of each 32-bit TMEM word holds k-block 4g + j's
+// scale; the MMA picks it with the instruction's scale-factor IDs.
 constexpr int ACC_COLS_UP = 2 * NT, ACC_COLS_DOWN = NT;
 constexpr int SF_COL0 = 2 * ACC_COLS_UP;
+// A slot is rewritten SF_SLOTS groups later, at least SF_SLOTS k-blocks on:
+// by then the MMAs that read it are complete (the MMA thread has passed the
+// full barrier of a stage the producer refilled after their commit), as long
+// as SF_SLOTS exceeds the deeper ring's 9 stages.
+constexpr int SF_SLOTS = 10;
 template <bool UP> struct SfCols {
-  static constexpr int PER_STAGE = UP ? 12 : 8;
+  static constexpr int PER_SLOT = UP ? 12 : 8;
 };
-static_assert(SF_COL0 + 5 * 12 <= (int)FTMEM && SF_COL0 + 9 * 8 <= (int)FTMEM, "TMEM columns");
+static_assert(SF_COL0 + SF_SLOTS * 12 <= (int)FTMEM, "TMEM columns");
 // Per stage in shared memory, the scale-factor bytes the MMA thread copies to
-// TMEM (tcgen05.cp 32x128b.warpx4): 512 bytes each for SFA (w1), SFA (w3, UP)
-// and SFB, row r = TMEM lane r of each of the four sub-partitions.
+// TMEM (tcgen05.cp 32x128b.warpx4) when the stage starts a group: 512 bytes
+// each for SFA (w1), SFA (w3, UP) and SFB, row r = TMEM lane r of each of the
+// four sub-partitions.
 constexpr int SF_BYTES = 512;
-constexpr int SF_STAGE_MAX = 3 * SF_BYTES;
 constexpr int SC_SLOT = NT * MAX_KB * 4;      // one tile's token scales (8 KB)
 // alignment slack, stages, the stages' scale-factor bytes, barriers (512), P
 // and off, 16 bytes to align the scale slots, the two scale slots, the
@@ -80,10 +86,11 @@ constexpr size_t FSMEM = 1024 + (size_t)RING_BYTES + 9 * 2 * SF_BYTES + 512 +
 static_assert(5 * 3 * SF_BYTES <= 9 * 2 * SF_BYTES, "UP scale-factor bytes");
 
 // kind::mxf8f6f4 block-scaled instruction descriptor: e4m3 A and B, both
-// K-major, fp32 accumulator, UE8M0 scale factors (bit 23), scale-factor byte
-// 0 of A's and B's TMEM words (bits 29-30, 4-5), M x N.
-__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N) {
-  return ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+// K-major, fp32 accumulator, UE8M0 scale factors (bit 23), byte `sf` of A's
+// and B's TMEM scale words (bits 29-30 and 4-5), M x N.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sf) {
+  return (sf << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+         (sf << 29);
 }
 
 // D[M x N] (+)= (A * 2^SFA) (B * 2^SFB)^T over K = 32: one UE8M0 scale per row
@@ -187,8 +194,6 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i) {
   }
   return t;
 }
-
-__device__ __forceinline__ int round16(int r) { return (r + 15) & ~15; }
 
 // Row stride, in floats, of the activation scales inside the layer: K/128
 // rounded up to a multiple of 4, so every row starts 16-byte aligned and a
@@ -389,18 +394,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        // the stage's scale factors (the stage's previous MMAs, and the copies
-        // to TMEM before them, are complete: empty[s] came from their commit)
-        uint8_t* sf = sfs + s * SF_STAGE;
-        const uint32_t b1 = __shfl_sync(0xffffffffu, kb < 32 ? w1a : w1b, kb & 31) * 0x01010101u;
-        *reinterpret_cast<uint4*>(sf + lane * 16) = make_uint4(b1, b1, b1, b1);
-        if (UP) {
-          const uint32_t b3 = __shfl_sync(0xffffffffu, kb < 32 ? w3a : w3b, kb & 31) * 0x01010101u;
-          *reinterpret_cast<uint4*>(sf + SF_BYTES + lane * 16) = make_uint4(b3, b3, b3, b3);
+        if ((kb & 3) == 0) {
+          // a group's first stage: the scale factors of k-blocks kb .. kb + 3,
+          // byte j for kb + j (bytes past the tile's k-blocks are not read).
+          // The stage's previous MMAs, and the copies to TMEM before them, are
+          // complete: empty[s] came from their commit.
+          uint8_t* sf = sfs + s * SF_STAGE;
+          uint32_t p1 = 0, p3 = 0, pt = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int k = kb + j;
+            p1 |= __shfl_sync(0xffffffffu, k < 32 ? w1a : w1b, k & 31) << (8 * j);
+            if (UP) p3 |= __shfl_sync(0xffffffffu, k < 32 ? w3a : w3b, k & 31) << (8 * j);
+            pt |= (lane < t.rows && k < kb_n ? ue8m0(ts[lane * kbp + k]) : 127u) << (8 * j);
+          }
+          *reinterpret_cast<uint4*>(sf + lane * 16) = make_uint4(p1, p1, p1, p1);
+          if (UP) *reinterpret_cast<uint4*>(sf + SF_BYTES + lane * 16) = make_uint4(p3, p3, p3, p3);
+          *reinterpret_cast<uint4*>(sf + (UP ? 2 : 1) * SF_BYTES + lane * 16) = make_uint4(pt, 0u, 0u, 0u);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        const uint32_t bt = (lane < t.rows ? ue8m0(ts[lane * kbp + kb]) : 127u) * 0x01010101u;
-        *reinterpret_cast<uint4*>(sf + (UP ? 2 : 1) * SF_BYTES + lane * 16) = make_uint4(bt, bt, bt, bt);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         uint8_t* sa = tiles + s * FSTAGE;
         uint8_t* sw = sa + A_BYTES;
@@ -430,15 +442,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // Per stage: the scale factors to TMEM (tcgen05.cp, ordered before the
-    // MMAs this thread issues after it), then four K = 32 block-scaled MMAs
-    // (eight for UP: w1 and w3) into the tile's accumulator, which sums the
-    // whole K; one commit per tile hands it to the epilogue.
+    // Per group of four stages: the scale factors to TMEM (tcgen05.cp,
+    // ordered before the MMAs this thread issues after it); per stage four
+    // K = 32 block-scaled MMAs (eight for UP: w1 and w3) into the tile's
+    // accumulator, which sums the whole K, reading byte kb % 4 of the scale
+    // words; one commit per tile hands it to the epilogue.
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
+      int s = 0, groups = 0;
+      uint32_t ph = 0, tsa = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_mx_e4m3(QB, NT);
       for (int i = blockIdx.x, lt = 0; ok && i < S.total; i += gridDim.x, ++lt) {
         const Tile t = decode(S, i);
         const int kb_n = g.kdim[t.kind] / QB;
@@ -451,18 +463,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           tc_fence_after();
           const uint32_t a0 = smem_u32(tiles + s * FSTAGE);
           const uint32_t w0 = a0 + A_BYTES;
-          const uint32_t sf0 = smem_u32(sfs + s * SF_STAGE);
-          const uint32_t tsa = tmem_base + (uint32_t)(SF_COL0 + s * SfCols<UP>::PER_STAGE);
-          const uint32_t tsb = tsa + (UP ? 8 : 4);
-          tmem_cp_sf(tsa, sdesc_sf(sf0));
-          if (UP) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
-          tmem_cp_sf(tsb, sdesc_sf(sf0 + (UP ? 2 : 1) * SF_BYTES));
+          if ((kb & 3) == 0) {
+            const uint32_t sf0 = smem_u32(sfs + s * SF_STAGE);
+            tsa = tmem_base + (uint32_t)(SF_COL0 + (groups % SF_SLOTS) * SfCols<UP>::PER_SLOT);
+            ++groups;
+            tmem_cp_sf(tsa, sdesc_sf(sf0));
+            if (UP) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
+            tmem_cp_sf(tsa + (UP ? 8 : 4), sdesc_sf(sf0 + (UP ? 2 : 1) * SF_BYTES));
+          }
+          // byte j = kb % 4 of the words: in the instruction descriptor and,
+          // as the byte address, in the top two bits of the TMEM addresses
+          const uint32_t j = (uint32_t)(kb & 3);
+          const uint32_t idesc = idesc_mx_e4m3(QB, NT, j);
+          const uint32_t sfa1 = tsa | (j << 30), sfa3 = (tsa + 4) | (j << 30);
+          const uint32_t sfb = (tsa + (UP ? 8 : 4)) | (j << 30);
 #pragma unroll
           for (int kk = 0; kk < QB / 32; ++kk) {
             const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            mma_mx(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, tsa, tsb, acc);
-            if (UP) mma_mx(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc, tsa + 4,
-                           tsb, acc);
+            mma_mx(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, sfa1, sfb, acc);
+            if (UP) mma_mx(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc, sfa3,
+                           sfb, acc);
           }
           tc_commit(&empty[s]);
           if (++s == FSTAGES) { s = 0; ph ^= 1; }
