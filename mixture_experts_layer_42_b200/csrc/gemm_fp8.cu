@@ -45,11 +45,13 @@ constexpr int W_BYTES = QB * QB;               // 16 KB per weight tile
 // Stages: UP carries the w1 and w3 tiles (36 KB, 5 stages), DOWN one w2 tile
 // (20 KB, 9 stages), so both keep ~160-180 KB of weights in flight per SM.
 template <bool UP> struct Ring {
-  static constexpr int STAGES = UP ? 5 : 9;
-  static constexpr int BYTES = A_BYTES + (UP ? 2 : 1) * W_BYTES;
+  static constexpr int KPS = UP ? 1 : 2;   // 128-deep k-blocks per stage
+  static constexpr int STAGES = UP ? 5 : 4;
+  static constexpr int BYTES = KPS * (A_BYTES + (UP ? 2 : 1) * W_BYTES);
 };
 constexpr int RING_BYTES = 9 * (A_BYTES + W_BYTES);  // the larger of the two rings (184 KB)
-static_assert(5 * (A_BYTES + 2 * W_BYTES) <= RING_BYTES, "UP ring");
+static_assert(Ring<true>::STAGES * Ring<true>::BYTES <= RING_BYTES, "UP ring");
+static_assert(Ring<false>::STAGES * Ring<false>::BYTES <= RING_BYTES, "DOWN ring");
 constexpr int NTHREADS = 192;
 constexpr uint32_t FTMEM = 256;
 constexpr int MAXE = 1024;
@@ -66,12 +68,13 @@ constexpr int SF_COL0 = 2 * ACC_COLS_UP;
 // A slot is rewritten SF_SLOTS groups later, at least SF_SLOTS k-blocks on:
 // by then the MMAs that read it are complete (the MMA thread has passed the
 // full barrier of a stage the producer refilled after their commit), as long
-// as SF_SLOTS exceeds the deeper ring's 9 stages.
+// as SF_SLOTS exceeds either ring's stages.
 constexpr int SF_SLOTS = 10;
 template <bool UP> struct SfCols {
   static constexpr int PER_SLOT = UP ? 12 : 8;
 };
 static_assert(SF_COL0 + SF_SLOTS * 12 <= (int)FTMEM, "TMEM columns");
+static_assert(SF_SLOTS > 5, "scale-factor slots outlive the ring");
 // Per stage in shared memory, the scale-factor bytes the MMA thread copies to
 // TMEM (tcgen05.cp 32x128b.warpx4) when the stage starts a group: 512 bytes
 // each for SFA (w1), SFA (w3, UP) and SFB, row r = TMEM lane r of each of the
@@ -165,16 +168,16 @@ struct Sched {
   int E, nb0, nb1, ch_sh, routed, total, t_shared;
 };
 
-__device__ __forceinline__ Tile decode(const Sched& S, int i) {
+// Tile i. `hint` is the expert of the caller's previous routed tile: a thread
+// visits its tiles in increasing order, so the expert only moves forward (a
+// few steps from the hint instead of a binary search per tile).
+__device__ __forceinline__ Tile decode(const Sched& S, int i, int& hint) {
   Tile t;
   if (i < S.routed) {
     const int q = i / S.nb0;
-    int lo = 0, hi = S.E;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (S.P[mid] <= q) lo = mid; else hi = mid;
-    }
-    const int e = lo;
+    int e = hint;
+    while (S.P[e + 1] <= q) ++e;
+    hint = e;
     const int mt = S.P[e + 1] - S.P[e];
     const int l = i - S.nb0 * S.P[e];
     const int nb = l / mt, c = l % mt;
@@ -330,10 +333,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // its row of each stage's scale-factor bytes: the weight block's scale
     // (the same for all 128 weight rows of the tile) and its token's.
     int s = 0, issued = 0, scopies = 0;
+    int hint = 0, hint_next = 0;            // experts of the last tile decoded, this and next
     uint32_t ph = 0;
     bool ok = true;
     if (lane == 0 && (int)blockIdx.x < S.total) {   // the first tile's token scales
-      const Tile t0 = decode(S, blockIdx.x);
+      int h0 = 0;
+      const Tile t0 = decode(S, blockIdx.x, h0);
       const int kbp = scale_stride(g.kdim[t0.kind]);
       const uint32_t bytes = (uint32_t)(t0.rows * kbp * 4);
       mbar_expect_tx(&sfull[0], bytes);
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       ++scopies;
     }
     for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
-      const Tile t = decode(S, i);
+      const Tile t = decode(S, i, hint);
       const int kb_n = g.kdim[t.kind] / QB;
       const int kbp = scale_stride(g.kdim[t.kind]);
       const int slot = lt & 1;
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
       }
       if (lane == 0 && i + (int)gridDim.x < S.total) {
-        const Tile tn = decode(S, i + gridDim.x);
+        const Tile tn = decode(S, i + gridDim.x, hint_next);
         const int kbpn = scale_stride(g.kdim[tn.kind]);
         const uint32_t bytes = (uint32_t)(tn.rows * kbpn * 4);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       // load of NT rows (rows past a tile's tokens are multiplied and not
       // stored; past the tensor's end they read zeros)
       const bool gath = UP && t.kind == 0;
-      const uint32_t tx = (uint32_t)(NT * QB + (UP ? 2 : 1) * W_BYTES);
+      constexpr int KPS = Ring<UP>::KPS;
       int r[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -390,7 +395,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         if (j < t.rows) a = (UP && t.kind == 0 && g.src != nullptr) ? g.src[row] : row;
         r[q] = a;
       }
-      for (int kb = 0; kb < kb_n; ++kb) {
+      for (int kb = 0; kb < kb_n; kb += KPS) {
+        const int nk = kb_n - kb < KPS ? kb_n - kb : KPS;   // k-blocks in this stage
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
@@ -414,13 +420,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
+        // stage layout: the KPS token tiles, then per k-block its weight tile(s)
         uint8_t* sa = tiles + s * FSTAGE;
-        uint8_t* sw = sa + A_BYTES;
         if (lane == 0) {
-          mbar_expect_tx(&full[s], tx);
-          tma_load_3d(sw, &g.tmW1[t.kind], &full[s], kb * QB, t.n0, t.e);
-          if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], kb * QB, t.n0, t.e);
-          if (!gath) tma_load_2d(sa, &g.tmAt[t.kind], &full[s], kb * QB, t.row0);
+          mbar_expect_tx(&full[s], (uint32_t)(nk * (NT * QB + (UP ? 2 : 1) * W_BYTES)));
+          for (int q = 0; q < nk; ++q) {
+            uint8_t* sw = sa + KPS * A_BYTES + q * (UP ? 2 : 1) * W_BYTES;
+            tma_load_3d(sw, &g.tmW1[t.kind], &full[s], (kb + q) * QB, t.n0, t.e);
+            if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], (kb + q) * QB, t.n0, t.e);
+            if (!gath) tma_load_2d(sa + q * A_BYTES, &g.tmAt[t.kind], &full[s], (kb + q) * QB, t.row0);
+          }
         }
         __syncwarp();
         if (gath && lane < NT / 4)
@@ -448,21 +457,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // accumulator, which sums the whole K, reading byte kb % 4 of the scale
     // words; one commit per tile hands it to the epilogue.
     if (lane == 0) {
-      int s = 0, groups = 0;
+      int s = 0, groups = 0, hint = 0;
       uint32_t ph = 0, tsa = 0;
       bool ok = true;
       for (int i = blockIdx.x, lt = 0; ok && i < S.total; i += gridDim.x, ++lt) {
-        const Tile t = decode(S, i);
+        const Tile t = decode(S, i, hint);
         const int kb_n = g.kdim[t.kind] / QB;
         const int b = lt & 1;
         if (!mbar_wait(&tempty[b], ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag, g.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(b * ACC_COLS);
-        for (int kb = 0; kb < kb_n; ++kb) {
+        constexpr int KPS = Ring<UP>::KPS;
+        for (int kb = 0; kb < kb_n; kb += KPS) {
+          const int nk = kb_n - kb < KPS ? kb_n - kb : KPS;
           if (!mbar_wait(&full[s], ph, abort_flag, g.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(tiles + s * FSTAGE);
-          const uint32_t w0 = a0 + A_BYTES;
           if ((kb & 3) == 0) {
             const uint32_t sf0 = smem_u32(sfs + s * SF_STAGE);
             tsa = tmem_base + (uint32_t)(SF_COL0 + (groups % SF_SLOTS) * SfCols<UP>::PER_SLOT);
@@ -471,18 +481,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
             if (UP) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
             tmem_cp_sf(tsa + (UP ? 8 : 4), sdesc_sf(sf0 + (UP ? 2 : 1) * SF_BYTES));
           }
-          // byte j = kb % 4 of the words: in the instruction descriptor and,
-          // as the byte address, in the top two bits of the TMEM addresses
-          const uint32_t j = (uint32_t)(kb & 3);
-          const uint32_t idesc = idesc_mx_e4m3(QB, NT, j);
-          const uint32_t sfa1 = tsa | (j << 30), sfa3 = (tsa + 4) | (j << 30);
-          const uint32_t sfb = (tsa + (UP ? 8 : 4)) | (j << 30);
+          for (int q = 0; q < nk; ++q) {
+            const uint32_t aq = a0 + q * A_BYTES;
+            const uint32_t wq = a0 + KPS * A_BYTES + q * (UP ? 2 : 1) * W_BYTES;
+            // byte j = (kb + q) % 4 of the words: in the instruction
+            // descriptor and, as the byte address, in the top two bits of the
+            // TMEM addresses
+            const uint32_t j = (uint32_t)((kb + q) & 3);
+            const uint32_t idesc = idesc_mx_e4m3(QB, NT, j);
+            const uint32_t sfa1 = tsa | (j << 30), sfa3 = (tsa + 4) | (j << 30);
+            const uint32_t sfb = (tsa + (UP ? 8 : 4)) | (j << 30);
 #pragma unroll
-          for (int kk = 0; kk < QB / 32; ++kk) {
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            mma_mx(d, sdesc(w0 + kk * 32), sdesc(a0 + kk * 32), idesc, sfa1, sfb, acc);
-            if (UP) mma_mx(d + NT, sdesc(w0 + W_BYTES + kk * 32), sdesc(a0 + kk * 32), idesc, sfa3,
-                           sfb, acc);
+            for (int kk = 0; kk < QB / 32; ++kk) {
+              const uint32_t acc = (kb + q > 0 || kk > 0) ? 1u : 0u;
+              mma_mx(d, sdesc(wq + kk * 32), sdesc(aq + kk * 32), idesc, sfa1, sfb, acc);
+              if (UP) mma_mx(d + NT, sdesc(wq + W_BYTES + kk * 32), sdesc(aq + kk * 32), idesc, sfa3,
+                             sfb, acc);
+            }
           }
           tc_commit(&empty[s]);
           if (++s == FSTAGES) { s = 0; ph ^= 1; }
@@ -498,10 +513,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // The tile's fp32 sums (scales already applied by the tensor core): a
     // TMEM lane is a weight row f, a column a token.
     const int quad = warp & 3;
+    int hint = 0;
     const int f = quad * 32 + lane;      // this thread's weight row (TMEM lane) in the tile
     const int et = threadIdx.x - 64;     // 0..127 among the epilogue threads
     for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
-      const Tile t = decode(S, i);
+      const Tile t = decode(S, i, hint);
       const int b = lt & 1;
       bool ok;
       {
