@@ -11,8 +11,9 @@
 // kernel); h = silu(w1 x) * (w3 x) is quantized by the up-projection's
 // epilogue; each expert's output is bf16, as on the bf16 path.
 //
-// Tiles put the weights on the MMA's M side (128 rows: one scale block) and
-// up to NT = 32 tokens of one expert on its N side, so a decode batch (a few
+// Tiles put the weights on the MMA's M side (MMAs of 128 rows: one scale
+// block; two per stage, UP's w1 and w3 rows or 256 of DOWN's w2 rows) and up
+// to NT = 32 tokens of one expert on its N side, so a decode batch (a few
 // tokens per expert) does little MMA work while it streams the active
 // experts' weights at half the bytes of bf16. Every MMA is block-scaled: per
 // 32-deep slice of K it multiplies each weight row by its UE8M0 scale and each
@@ -44,10 +45,18 @@ constexpr int A_BYTES = NT * QB;               // 4 KB of token rows
 constexpr int W_BYTES = QB * QB;               // 16 KB per weight tile
 // Stages: UP carries the w1 and w3 tiles (36 KB, 5 stages), DOWN one w2 tile
 // (20 KB, 9 stages), so both keep ~160-180 KB of weights in flight per SM.
+// A stage holds KPS k-blocks: per k-block the tile's token rows and its two
+// 128-row weight tiles (UP: w1 and w3; DOWN: two consecutive blocks of w2's
+// rows, so a DOWN tile covers 256 output features).
 template <bool UP> struct Ring {
-  static constexpr int KPS = UP ? 1 : 2;   // 128-deep k-blocks per stage
-  static constexpr int STAGES = UP ? 5 : 4;
-  static constexpr int BYTES = KPS * (A_BYTES + (UP ? 2 : 1) * W_BYTES);
+  static constexpr int KPS = 1;   // 128-deep k-blocks per stage
+  static constexpr int STAGES = 5;
+  static constexpr int BYTES = KPS * (A_BYTES + 2 * W_BYTES);
+};
+// Output features per tile: UP 128 (the w1 rows, with the w3 rows beside
+// them), DOWN 256.
+template <bool UP> struct TileN {
+  static constexpr int BN = UP ? QB : 2 * QB;
 };
 constexpr int RING_BYTES = 9 * (A_BYTES + W_BYTES);  // the larger of the two rings (184 KB)
 static_assert(Ring<true>::STAGES * Ring<true>::BYTES <= RING_BYTES, "UP ring");
@@ -63,15 +72,15 @@ constexpr int MAX_KB = 64;                     // k-blocks per tile (K <= 8192)
 // (SFA; w1 and w3 each for UP) and 4 for the tokens' (SFB; only the first is
 // read at N = 32). Byte j of each 32-bit TMEM word holds k-block 4g + j's
 // scale; the MMA picks it with the instruction's scale-factor IDs.
-constexpr int ACC_COLS_UP = 2 * NT, ACC_COLS_DOWN = NT;
-constexpr int SF_COL0 = 2 * ACC_COLS_UP;
+constexpr int ACC_COLS = 2 * NT;
+constexpr int SF_COL0 = 2 * ACC_COLS;
 // A slot is rewritten SF_SLOTS groups later, at least SF_SLOTS k-blocks on:
 // by then the MMAs that read it are complete (the MMA thread has passed the
 // full barrier of a stage the producer refilled after their commit), as long
 // as SF_SLOTS exceeds either ring's stages.
 constexpr int SF_SLOTS = 10;
 template <bool UP> struct SfCols {
-  static constexpr int PER_SLOT = UP ? 12 : 8;
+  static constexpr int PER_SLOT = 12;
 };
 static_assert(SF_COL0 + SF_SLOTS * 12 <= (int)FTMEM, "TMEM columns");
 static_assert(SF_SLOTS > 5, "scale-factor slots outlive the ring");
@@ -165,7 +174,7 @@ struct Tile {
 struct Sched {
   const int32_t* P;
   const int32_t* off;
-  int E, nb0, nb1, ch_sh, routed, total, t_shared;
+  int E, nb0, nb1, ch_sh, routed, total, t_shared, bn;
 };
 
 // Tile i. `hint` is the expert of the caller's previous routed tile: a thread
@@ -185,7 +194,7 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i, int& hint) {
     t.e = e;
     t.row0 = S.off[e] + c * NT;
     t.rows = min(NT, S.off[e + 1] - t.row0);
-    t.n0 = nb * QB;
+    t.n0 = nb * S.bn;
   } else {
     const int l = i - S.routed;
     const int nb = l / S.ch_sh, c = l % S.ch_sh;
@@ -193,7 +202,7 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i, int& hint) {
     t.e = 0;
     t.row0 = c * NT;
     t.rows = min(NT, S.t_shared - t.row0);
-    t.n0 = nb * QB;
+    t.n0 = nb * S.bn;
   }
   return t;
 }
@@ -243,10 +252,9 @@ template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  constexpr int ACC_COLS = UP ? ACC_COLS_UP : ACC_COLS_DOWN;
   constexpr int FSTAGES = Ring<UP>::STAGES;
   constexpr int FSTAGE = Ring<UP>::BYTES;
-  constexpr int SF_STAGE = (UP ? 3 : 2) * SF_BYTES;   // SFA (w1), [SFA (w3)], SFB
+  constexpr int SF_STAGE = 3 * SF_BYTES;   // SFA (first weight tile), SFA (second), SFB
   uint8_t* sfs = tiles + RING_BYTES;                  // [FSTAGES][SF_STAGE]
   uint64_t* full = reinterpret_cast<uint64_t*>(sfs + 9 * 2 * SF_BYTES);
   uint64_t* empty = full + FSTAGES;
@@ -319,8 +327,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
   S.P = P;
   S.off = off;
   S.E = E;
-  S.nb0 = g.n_out[0] / QB;
-  S.nb1 = g.t_shared > 0 ? g.n_out[1] / QB : 0;
+  S.bn = TileN<UP>::BN;
+  S.nb0 = (g.n_out[0] + S.bn - 1) / S.bn;
+  S.nb1 = g.t_shared > 0 ? (g.n_out[1] + S.bn - 1) / S.bn : 0;
   S.ch_sh = (g.t_shared + NT - 1) / NT;
   S.t_shared = g.t_shared;
   S.routed = S.nb0 * P[E];
@@ -350,14 +359,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       const int kb_n = g.kdim[t.kind] / QB;
       const int kbp = scale_stride(g.kdim[t.kind]);
       const int slot = lt & 1;
+      // the second weight tile: UP w3's rows, DOWN the next 128 rows of w2
+      // (none in a DOWN tile at the end of an odd number of row blocks)
+      const bool two = UP || t.n0 + QB < g.n_out[t.kind];
       // the tile's weight scales as UE8M0 bytes, k-blocks lane and lane + 32
       const int nbw = g.n_out[t.kind] / QB;
       const float* pw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
       const uint32_t w1a = lane < kb_n ? ue8m0(__ldg(pw1 + lane)) : 127u;
       const uint32_t w1b = lane + 32 < kb_n ? ue8m0(__ldg(pw1 + lane + 32)) : 127u;
       uint32_t w3a = 127u, w3b = 127u;
-      if (UP) {
-        const float* pw3 = g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
+      if (two) {
+        const float* pw3 = UP ? g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n : pw1 + kb_n;
         w3a = lane < kb_n ? ue8m0(__ldg(pw3 + lane)) : 127u;
         w3b = lane + 32 < kb_n ? ue8m0(__ldg(pw3 + lane + 32)) : 127u;
       }
@@ -411,23 +423,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           for (int j = 0; j < 4; ++j) {
             const int k = kb + j;
             p1 |= __shfl_sync(0xffffffffu, k < 32 ? w1a : w1b, k & 31) << (8 * j);
-            if (UP) p3 |= __shfl_sync(0xffffffffu, k < 32 ? w3a : w3b, k & 31) << (8 * j);
+            p3 |= __shfl_sync(0xffffffffu, k < 32 ? w3a : w3b, k & 31) << (8 * j);
             pt |= (lane < t.rows && k < kb_n ? ue8m0(ts[lane * kbp + k]) : 127u) << (8 * j);
           }
           *reinterpret_cast<uint4*>(sf + lane * 16) = make_uint4(p1, p1, p1, p1);
-          if (UP) *reinterpret_cast<uint4*>(sf + SF_BYTES + lane * 16) = make_uint4(p3, p3, p3, p3);
-          *reinterpret_cast<uint4*>(sf + (UP ? 2 : 1) * SF_BYTES + lane * 16) = make_uint4(pt, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sf + SF_BYTES + lane * 16) = make_uint4(p3, p3, p3, p3);
+          *reinterpret_cast<uint4*>(sf + 2 * SF_BYTES + lane * 16) = make_uint4(pt, 0u, 0u, 0u);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
         __syncwarp();
         // stage layout: the KPS token tiles, then per k-block its weight tile(s)
         uint8_t* sa = tiles + s * FSTAGE;
         if (lane == 0) {
-          mbar_expect_tx(&full[s], (uint32_t)(nk * (NT * QB + (UP ? 2 : 1) * W_BYTES)));
+          mbar_expect_tx(&full[s], (uint32_t)(nk * (NT * QB + (two ? 2 : 1) * W_BYTES)));
           for (int q = 0; q < nk; ++q) {
-            uint8_t* sw = sa + KPS * A_BYTES + q * (UP ? 2 : 1) * W_BYTES;
+            uint8_t* sw = sa + KPS * A_BYTES + q * 2 * W_BYTES;
             tma_load_3d(sw, &g.tmW1[t.kind], &full[s], (kb + q) * QB, t.n0, t.e);
             if (UP) tma_load_3d(sw + W_BYTES, &g.tmW3[t.kind], &full[s], (kb + q) * QB, t.n0, t.e);
+            else if (two) tma_load_3d(sw + W_BYTES, &g.tmW1[t.kind], &full[s], (kb + q) * QB, t.n0 + QB, t.e);
             if (!gath) tma_load_2d(sa + q * A_BYTES, &g.tmAt[t.kind], &full[s], (kb + q) * QB, t.row0);
           }
         }
@@ -453,9 +466,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // ---------------------------------------------------------------- MMA issuer
     // Per group of four stages: the scale factors to TMEM (tcgen05.cp,
     // ordered before the MMAs this thread issues after it); per stage four
-    // K = 32 block-scaled MMAs (eight for UP: w1 and w3) into the tile's
-    // accumulator, which sums the whole K, reading byte kb % 4 of the scale
-    // words; one commit per tile hands it to the epilogue.
+    // K = 32 block-scaled MMAs per weight tile (two tiles: UP w1 and w3, DOWN
+    // two row blocks of w2) into the tile's accumulator, which sums the whole
+    // K, reading byte kb % 4 of the scale words; one commit per tile hands it
+    // to the epilogue.
     if (lane == 0) {
       int s = 0, groups = 0, hint = 0;
       uint32_t ph = 0, tsa = 0;
@@ -463,6 +477,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       for (int i = blockIdx.x, lt = 0; ok && i < S.total; i += gridDim.x, ++lt) {
         const Tile t = decode(S, i, hint);
         const int kb_n = g.kdim[t.kind] / QB;
+        const bool two = UP || t.n0 + QB < g.n_out[t.kind];
         const int b = lt & 1;
         if (!mbar_wait(&tempty[b], ((uint32_t)(lt >> 1) & 1) ^ 1, abort_flag, g.err)) { ok = false; break; }
         tc_fence_after();
@@ -478,25 +493,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
             tsa = tmem_base + (uint32_t)(SF_COL0 + (groups % SF_SLOTS) * SfCols<UP>::PER_SLOT);
             ++groups;
             tmem_cp_sf(tsa, sdesc_sf(sf0));
-            if (UP) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
-            tmem_cp_sf(tsa + (UP ? 8 : 4), sdesc_sf(sf0 + (UP ? 2 : 1) * SF_BYTES));
+            if (two) tmem_cp_sf(tsa + 4, sdesc_sf(sf0 + SF_BYTES));
+            tmem_cp_sf(tsa + 8, sdesc_sf(sf0 + 2 * SF_BYTES));
           }
           for (int q = 0; q < nk; ++q) {
             const uint32_t aq = a0 + q * A_BYTES;
-            const uint32_t wq = a0 + KPS * A_BYTES + q * (UP ? 2 : 1) * W_BYTES;
+            const uint32_t wq = a0 + KPS * A_BYTES + q * 2 * W_BYTES;
             // byte j = (kb + q) % 4 of the words: in the instruction
             // descriptor and, as the byte address, in the top two bits of the
             // TMEM addresses
             const uint32_t j = (uint32_t)((kb + q) & 3);
             const uint32_t idesc = idesc_mx_e4m3(QB, NT, j);
             const uint32_t sfa1 = tsa | (j << 30), sfa3 = (tsa + 4) | (j << 30);
-            const uint32_t sfb = (tsa + (UP ? 8 : 4)) | (j << 30);
+            const uint32_t sfb = (tsa + 8) | (j << 30);
 #pragma unroll
             for (int kk = 0; kk < QB / 32; ++kk) {
               const uint32_t acc = (kb + q > 0 || kk > 0) ? 1u : 0u;
               mma_mx(d, sdesc(wq + kk * 32), sdesc(aq + kk * 32), idesc, sfa1, sfb, acc);
-              if (UP) mma_mx(d + NT, sdesc(wq + W_BYTES + kk * 32), sdesc(aq + kk * 32), idesc, sfa3,
-                             sfb, acc);
+              if (two) mma_mx(d + NT, sdesc(wq + W_BYTES + kk * 32), sdesc(aq + kk * 32), idesc, sfa3,
+                              sfb, acc);
             }
           }
           tc_commit(&empty[s]);
@@ -518,6 +533,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     const int et = threadIdx.x - 64;     // 0..127 among the epilogue threads
     for (int i = blockIdx.x, lt = 0; i < S.total; i += gridDim.x, ++lt) {
       const Tile t = decode(S, i, hint);
+      const bool two = UP || t.n0 + QB < g.n_out[t.kind];
       const int b = lt & 1;
       bool ok;
       {
@@ -525,7 +541,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         if (lane == 0) w = mbar_wait(&tfull[b], (uint32_t)(lt >> 1) & 1, abort_flag, g.err) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, w, 0) != 0;
       }
-      float sa[NT], sb[UP ? NT : 1];
+      float sa[NT], sb[NT];
       if (ok) {
         tc_fence_after();
         const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * ACC_COLS);
@@ -535,7 +551,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) { sa[j] = __uint_as_float(r0[j]); sa[16 + j] = __uint_as_float(r1[j]); }
-        if (UP) {
+        if (two) {
           tmem_ld16(tb + NT, r0);
           tmem_ld16(tb + NT + 16, r1);
           tmem_wait_ld();
@@ -574,11 +590,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           }
         }
       } else {
+        // the tile's two row blocks: features n0 + f and n0 + 128 + f
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(g.out[t.kind]);
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-          if (j < t.rows)
-            out[(int64_t)(t.row0 + j) * g.n_out[t.kind] + t.n0 + f] = __float2bfloat16_rn(sa[j]);
+        for (int j = 0; j < NT; ++j) {
+          if (j < t.rows) {
+            __nv_bfloat16* o = out + (int64_t)(t.row0 + j) * g.n_out[t.kind] + t.n0 + f;
+            o[0] = __float2bfloat16_rn(sa[j]);
+            if (two) o[QB] = __float2bfloat16_rn(sb[j]);
+          }
+        }
       }
     }
   }
@@ -821,8 +842,9 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
     g.E = E;
     g.t_shared = sh ? (int)T : 0;
     g.err = err;
-    const int64_t bound = (int64_t)(n0 / QB) * ((Tk + NT - 1) / NT + E) +
-                          (sh ? (int64_t)(n1 / QB) * ((T + NT - 1) / NT) : 0);
+    const int bn = up ? TileN<true>::BN : TileN<false>::BN;   // output features per tile
+    const int64_t bound = (int64_t)((n0 + bn - 1) / bn) * ((Tk + NT - 1) / NT + E) +
+                          (sh ? (int64_t)((n1 + bn - 1) / bn) * ((T + NT - 1) / NT) : 0);
     const int grid = (int)(bound < num_sms ? bound : num_sms);
     if (grid > 0) {
       if (up) {
