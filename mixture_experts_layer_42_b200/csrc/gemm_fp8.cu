@@ -397,6 +397,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       // load of NT rows (rows past a tile's tokens are multiplied and not
       // stored; past the tensor's end they read zeros)
       const bool gath = UP && t.kind == 0;
+      // token rows brought in per k-block: a gathered tile only its rows,
+      // rounded up to 4 (the MMA's other token columns read whatever the
+      // stage held; their sums are not stored), a tile load all NT
+      const int a_rows_ld = gath ? ((t.rows + 3) & ~3) : NT;
       constexpr int KPS = Ring<UP>::KPS;
       int r[4];
 #pragma unroll
@@ -435,7 +439,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
         // stage layout: the KPS token tiles, then per k-block its weight tile(s)
         uint8_t* sa = tiles + s * FSTAGE;
         if (lane == 0) {
-          mbar_expect_tx(&full[s], (uint32_t)(nk * (NT * QB + (two ? 2 : 1) * W_BYTES)));
+          mbar_expect_tx(&full[s], (uint32_t)(nk * (a_rows_ld * QB + (two ? 2 : 1) * W_BYTES)));
           for (int q = 0; q < nk; ++q) {
             uint8_t* sw = sa + KPS * A_BYTES + q * 2 * W_BYTES;
             tma_load_3d(sw, &g.tmW1[t.kind], &full[s], (kb + q) * QB, t.n0, t.e);
@@ -445,7 +449,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
           }
         }
         __syncwarp();
-        if (gath && lane < NT / 4)
+        if (gath && lane < a_rows_ld / 4)
           tma_gather4(sa + lane * (4 * QB), &g.tmA[t.kind], &full[s], kb * QB, r[0], r[1], r[2], r[3]);
         ++issued;
         if (++s == FSTAGES) { s = 0; ph ^= 1; }
