@@ -232,21 +232,6 @@ __device__ __forceinline__ uint8_t to_e4m3(float v) {
 
 __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
 
-// Named barrier 1 over the four epilogue warps that also ORs a flag across
-// them, so that every warp takes the same abort decision before the next
-// barrier (a warp that left alone would leave the others waiting).
-__device__ __forceinline__ bool epi_sync_any(bool flag) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.or.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)flag)
-      : "memory");
-  return r != 0;
-}
 
 template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {

@@ -279,6 +279,22 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 
 // Operands of one grouped expert launch on the tensor cores: [0] routed
 // experts (A rows expert-contiguous, B stacked per expert), [1] the shared MLP.
+// Named barrier 1 over the four epilogue warps that also ORs a flag across
+// them, so that every warp takes the same abort decision before the next
+// barrier (a warp that left alone would leave the others waiting).
+__device__ __forceinline__ bool epi_sync_any(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag)
+      : "memory");
+  return r != 0;
+}
+
 struct TcArgs {
   CUtensorMap tmA[2];   // [0] routed A rows, [1] shared A rows; 2D {K, rows}
   CUtensorMap tmA64[2]; // the same with 64-row boxes (CTA-pair tail chunks)
