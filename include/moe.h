@@ -282,10 +282,13 @@ MOE_API moe_status moe_check_error(void* ws, void* stream);
 /* Static text for a status code. */
 MOE_API const char* moe_status_string(moe_status st);
 
-/* Number of kernels moe_forward launches for this config with the expert
- * kernel currently selected (moe_select_expert_kernel), for accounting: 9
- * for a bf16 layer on the default one-CTA tensor-core kernel (the expert GEMMs
- * use one kernel that writes their per-expert A maps), 8 otherwise. */
+/* Number of kernels moe_forward launches for T tokens of this config with the
+ * expert kernel currently selected (moe_select_expert_kernel), for
+ * accounting: router 2, dispatch 3 (1 for a batch of at most 4096 (token,
+ * slot) pairs over at most 512 experts that reads the token rows from x),
+ * the two expert GEMMs (plus one kernel that writes their per-expert A maps
+ * on the default one-CTA tensor-core kernel), combine 1: 7 for the
+ * DeepSeek-V3 decode batch, 9 for its prefill batch. */
 MOE_API int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T);
 
 /* moe_gate without a workspace. The pages have no counterpart of this call:

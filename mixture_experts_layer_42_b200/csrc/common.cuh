@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -25,6 +27,10 @@ __host__ __device__ inline T ceil_div(T a, T b) { return (a + b - 1) / b; }
 
 // Tokens per dispatch chunk (the unit of the stable counting sort).
 constexpr int kDispatchChunkTokens = 64;
+// Batches up to this many (token, slot) pairs over at most this many experts,
+// without a permuted copy of x, are dispatched by one kernel (one CTA).
+constexpr int kDispatchSmallPairs = 4096;
+constexpr int kDispatchSmallExperts = 512;
 
 // Router GEMM tile: 128 tokens x 64 experts, 32-deep k slices.
 constexpr int kRouterBM = 128;
@@ -212,7 +218,31 @@ struct GroupedArgs {
 // Records the next per-kernel timing event on `st` when moe_forward runs with
 // stage timing on (see moe_stage_timing_begin); a no-op otherwise. Every
 // launcher calls it right after each kernel it launches.
+// A launch on `st`, as a programmatic dependent of the kernel before it in the
+// stream when `pdl` (it may start once that kernel's CTAs have all executed
+// griddepcontrol.launch_dependents, and must griddepcontrol.wait before it
+// reads that kernel's output), else an ordinary launch.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 void stage_mark(cudaStream_t st);
+// Whether the small kernels of a forward may be launched as programmatic
+// dependents of the kernel before them (not while the stage timer records
+// events between the launches).
+bool pdl_ok();
 // Whether the stage timer is recording the current forward call.
 bool stage_timing_active();
 
@@ -259,6 +289,12 @@ struct DispatchPlace {
   void* x_perm;
 };
 cudaError_t launch_dispatch_place(const DispatchPlace& p, cudaStream_t st);
+// The whole dispatch of a small batch (dispatch_small_ok) in one launch:
+// counts, offsets, pos and src, the same values as the three-kernel path.
+bool dispatch_small_ok(const moe_config& c, int64_t T, const void* x_perm);
+cudaError_t launch_dispatch_small(const moe_config& c, int64_t T, const int32_t* idx,
+                                  int32_t* counts, int32_t* offsets, int32_t* pos, int32_t* src,
+                                  uint32_t* err, cudaStream_t st);
 cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, const int32_t* pos,
                            const float* weights, const void* s, void* y, cudaStream_t st);
 // Expert parallelism: one rank's fp32 share of y (pairs routed to its

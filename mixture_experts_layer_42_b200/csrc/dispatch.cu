@@ -18,6 +18,8 @@
 //                           (row slices, tokens): pos, src, and the copy of
 //                           x[t] into its k permuted rows with 16-byte loads
 //                           and stores (x is read once).
+//   dispatch_small_kernel   small batches without a copy: all of the above in
+//                           one CTA (one launch instead of three).
 #include "common.cuh"
 
 namespace moe {
@@ -198,6 +200,110 @@ dispatch_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restri
   }
 }
 
+// Small batches (T*k <= kDispatchSmallPairs, E <= kDispatchSmallExperts, no
+// permuted copy): the whole stable counting sort in one CTA of SW warps, the
+// steps of the three kernels above in one launch. Warp w ranks the pairs
+// [w * per_warp, (w + 1) * per_warp) in rounds of 32 (ranks within the warp
+// by __match_any_sync, in pair order), an exclusive scan over the warps per
+// expert and one over the experts give each pair its row.
+constexpr int SW = 16;
+__global__ void __launch_bounds__(SW * 32)
+dispatch_small_kernel(const int32_t* __restrict__ idx, int64_t T, int k, int E,
+                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                      int32_t* __restrict__ pos, int32_t* __restrict__ src, uint32_t* err) {
+  extern __shared__ int32_t hist[];  // [SW][E], then the expert offsets [E + 1]
+  int32_t* eoff = hist + SW * E;
+  __shared__ int32_t wsum[SW];
+  // a programmatic dependent of the selection: the kernel after it may
+  // launch now; idx is read after the selection's grid completes
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = threadIdx.x; i < SW * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int64_t n = T * k;
+  const int per_warp = (int)ceil_div<int64_t>(ceil_div<int64_t>(n, SW), 32) * 32;
+  const int rounds = per_warp / 32;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int rank[kDispatchSmallPairs / SW / 32];
+  int ex[kDispatchSmallPairs / SW / 32];
+#pragma unroll
+  for (int r = 0; r < kDispatchSmallPairs / SW / 32; ++r) {
+    rank[r] = -1;
+    ex[r] = -1;
+    if (r >= rounds) continue;
+    const int64_t q = (int64_t)warp * per_warp + r * 32 + lane;
+    int e = -2;  // past the pairs
+    if (q < n) {
+      e = idx[q];
+      if (e < 0 || e >= E) {
+        set_error(err, ERRBIT_BAD_INDEX);
+        e = -1;
+      }
+    }
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    int base = 0;
+    if (e >= 0) base = hist[warp * E + e];
+    __syncwarp();
+    if (e >= 0) {
+      if ((__ffs(same) - 1) == lane) hist[warp * E + e] = base + __popc(same);
+      rank[r] = base + __popc(same & lt_mask);
+      ex[r] = e;
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: exclusive scan over the warps, the count; then the exclusive
+  // scan of the counts over the experts (E <= blockDim.x)
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+#pragma unroll
+    for (int w = 0; w < SW; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += c;
+    }
+    counts[e] = run;
+  }
+  int incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int p = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += p;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < SW ? wsum[lane] : 0;
+    int vi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int p = __shfl_up_sync(0xffffffffu, vi, o);
+      if (lane >= o) vi += p;
+    }
+    if (lane < SW) wsum[lane] = vi - v;
+  }
+  __syncthreads();
+  const int excl = incl - run + wsum[warp];
+  if (e < E) {
+    offsets[e] = excl;
+    eoff[e] = excl;
+  }
+  if (e == E - 1) offsets[E] = excl + run;
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kDispatchSmallPairs / SW / 32; ++r) {
+    if (r >= rounds) continue;
+    const int64_t q = (int64_t)warp * per_warp + r * 32 + lane;
+    if (q >= n) continue;
+    int p = -1;
+    if (ex[r] >= 0) p = eoff[ex[r]] + hist[warp * E + ex[r]] + rank[r];
+    pos[q] = p;
+    if (p >= 0) src[p] = (int32_t)(q / k);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch_sort(const moe_config& c, int64_t T, const int32_t* idx,
@@ -241,10 +347,27 @@ cudaError_t launch_dispatch_place(const DispatchPlace& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+bool dispatch_small_ok(const moe_config& c, int64_t T, const void* x_perm) {
+  return x_perm == nullptr && T * c.topk <= kDispatchSmallPairs && c.n_routed <= kDispatchSmallExperts;
+}
+
+cudaError_t launch_dispatch_small(const moe_config& c, int64_t T, const int32_t* idx,
+                                  int32_t* counts, int32_t* offsets, int32_t* pos, int32_t* src,
+                                  uint32_t* err, cudaStream_t st) {
+  const size_t smem = ((size_t)SW * c.n_routed + c.n_routed + 1) * sizeof(int32_t);
+  return launch_pdl(pdl_ok(), dispatch_small_kernel, dim3(1), dim3(SW * 32), smem, st, idx, T,
+                    c.topk, c.n_routed, counts, offsets, pos, src, err);
+}
+
 cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
                             int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                             void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,
                             uint32_t* err, cudaStream_t st) {
+  if (dispatch_small_ok(c, T, x_perm)) {
+    cudaError_t e = launch_dispatch_small(c, T, idx, counts, offsets, pos, src, err, st);
+    for (int m = 0; m < 3; ++m) stage_mark(st);   // the timer's three dispatch intervals
+    return e;
+  }
   cudaError_t e =
       launch_dispatch_sort(c, T, idx, counts, offsets, chunk_hist, pos_local, n_chunks, err, st);
   if (e != cudaSuccess) return e;

@@ -46,8 +46,6 @@
 // what it has in flight, frees TMEM and returns.
 #include "tc_common.cuh"
 
-#include <utility>
-
 namespace moe {
 
 namespace {
@@ -84,9 +82,7 @@ struct Sched {
   int E, nt0, nt1, mt_sh, routed, total, t_shared, bn_out;
 };
 
-// Tile i: the shared expert's tiles come first (they need only x, so the
-// up-projection can run them while the dispatch that feeds the routed tiles
-// is still finishing), then the routed experts' tiles.
+// Tile i: the shared expert's tiles first, then the routed experts' tiles.
 __device__ __forceinline__ Tile decode(const Sched& S, int i) {
   Tile t;
   const int n_sh = S.total - S.routed;
@@ -184,6 +180,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    // Launched as a programmatic dependent of the kernel before it (the
+    // dispatch or the row-map kernel), this grid may be running before that
+    // one completes: wait for it before anything it wrote is read (the
+    // offsets here; src, the row maps and the tile counter after the
+    // __syncthreads below). Returns at once for an ordinary launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // m-tiles per expert and their exclusive prefix
     const int per = (E + 31) / 32;
     int lsum = 0;
@@ -244,7 +246,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool ok = true;
-    bool dep_done = false;
     TileQueue Q;
     const bool dyn = g.tile_ctr != nullptr;
     // the next tile is claimed a few k-blocks before the current one ends,
@@ -271,13 +272,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       }
       if (i >= S.total) break;
       const Tile t = decode(S, i);
-      if (t.kind == 0 && !dep_done) {
-        // the routed rows (their copy or src), their maps: written by the
-        // kernels this launch may have started alongside (programmatic
-        // dependent launch); returns at once otherwise
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        dep_done = true;
-      }
       const int kb_n = (g.kdim[t.kind] + BK - 1) / BK;
       const int kb_claim = kb_n > 4 ? kb_n - 4 : 0;
       const bool swap = swap_tail(t, g);
@@ -549,6 +543,12 @@ struct RowMapArgs {
 __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ RowMapArgs a,
                                                              const int32_t* __restrict__ offsets,
                                                              int E, int* tile_ctr) {
+  // the up-projection, a programmatic dependent of this kernel when the
+  // dispatch ran before it, may start now (it waits for this grid before its
+  // routed tiles); this kernel is itself a programmatic dependent of the
+  // dispatch, whose offsets it reads after that grid completes
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ __align__(128) CUtensorMap sm[8];
   const int w = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int which = blockIdx.y;
@@ -582,25 +582,6 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
 
 }  // namespace
 
-// A launch on `st`, as a programmatic dependent of the kernel before it in the
-// stream when `pdl` (it may start once that kernel's CTAs have all executed
-// griddepcontrol.launch_dependents, and must griddepcontrol.wait before it
-// reads that kernel's output), else an ordinary launch.
-template <typename... Params, typename... Args>
-static cudaError_t launch_k(bool pdl, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
-                            cudaStream_t st, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = pdl ? attr : nullptr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
 
 // Test hook state (moe_debug_stall_pipeline).
 static int g_stall = STALL_NONE;
@@ -619,8 +600,7 @@ cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, 
     a.maps[1] = static_cast<CUtensorMap*>(maps);
   }
   dim3 grid((unsigned)((E + 7) / 8), a_up != nullptr ? 2u : 1u);
-  build_row_maps_kernel<<<grid, 256, 0, st>>>(a, offsets, E, up_tile_ctr);
-  return cudaGetLastError();
+  return launch_pdl(pdl_ok(), build_row_maps_kernel, grid, dim3(256), 0, st, a, offsets, E, up_tile_ctr);
 }
 
 // A: routed rows [Tk, K0] (or, for UP, the token rows gx [gT, K0] gathered
@@ -730,13 +710,13 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
     e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = launch_k(pdl, grouped_tc_kernel<true>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
+    e = launch_pdl(pdl, grouped_tc_kernel<true>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
     if (e != cudaSuccess) return e;
   } else {
     e = cudaFuncSetAttribute(grouped_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = launch_k(pdl, grouped_tc_kernel<false>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
+    e = launch_pdl(pdl, grouped_tc_kernel<false>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, g);
     if (e != cudaSuccess) return e;
   }
   stage_mark(st);

@@ -96,15 +96,17 @@ moe_status bind_device(cudaStream_t s, const void* ptr) {
 // copy of x) or, when x_perm is null, are gathered from x through src. With
 // `place`, the dispatch's placement (pos, src, the copy) is launched here,
 // after the row maps (which need only the offsets) and right before the
-// up-projection, which then starts as a programmatic dependent of it (its
-// prologue and any shared-expert tiles, which come first and need only x, run
-// while the placement finishes; its producer waits for the placement's grid
-// before the first routed tile).
+// up-projection. With `dependent_up` (moe_forward), the up-projection is
+// launched as a programmatic dependent of the kernel before it (the placement,
+// or the row-map kernel after a one-kernel dispatch): its launch and setup
+// overlap that kernel's tail, and it waits for that grid before it reads
+// anything the dispatch wrote.
 moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const int32_t* src,
                        const int32_t* offsets, const void* w1, const void* w3, const void* w2,
                        const void* x, const void* ws1, const void* ws3, const void* ws2,
                        void* y_perm, void* s, void* h, void* hs, void* row_maps, uint32_t* err,
-                       cudaStream_t st, const DispatchPlace* place = nullptr) {
+                       cudaStream_t st, const DispatchPlace* place = nullptr,
+                       bool dependent_up = false) {
   const int64_t Tk = T * c.topk;
   const bool sh = c.shared_inter > 0;
   const bool tc = c.dtype == MOE_DT_BF16 && g_expert_kernel != MOE_EXPERT_KERNEL_SIMT;
@@ -128,8 +130,11 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
     }
     if (place != nullptr && launch_dispatch_place(*place, st) != cudaSuccess)
       return MOE_ERR_CUDA;
+    // a small batch's dispatch ran in one kernel before the row maps: close
+    // the timer's dispatch interval here (it then holds the row-map kernel)
+    if (place == nullptr && dependent_up) stage_mark(st);
     // (not while the stage timer records events between the launches)
-    const bool pdl = place != nullptr && kind == TC_ROWS && !stage_timing_active();
+    const bool pdl = (place != nullptr || dependent_up) && kind == TC_ROWS && !stage_timing_active();
     e = launch_grouped_tc(true, kind, Tk, sh ? T : 0, c.n_routed, x_perm, x, w1, w3, ws1, ws3,
                           c.moe_inter, c.dim, c.shared_inter, c.dim, h, hs, offsets, x,
                           x_perm ? nullptr : src, T, kind == TC_ROWS ? row_maps : nullptr, ctr, err,
@@ -143,6 +148,7 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
   }
   if (place != nullptr && launch_dispatch_place(*place, st) != cudaSuccess)
     return MOE_ERR_CUDA;
+  if (place == nullptr && dependent_up) stage_mark(st);
   GroupedArgs g;
   memset(&g, 0, sizeof(g));
   g.offsets = offsets;
@@ -217,6 +223,8 @@ bool fp8_shapes_ok(const moe_config& c) {
 }  // namespace
 
 bool stage_timing_active() { return g_timing.on && g_timing.in_forward; }
+
+bool pdl_ok() { return !stage_timing_active(); }
 
 void stage_mark(cudaStream_t st) {
   StageTiming& T = g_timing;
@@ -388,17 +396,27 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   const bool copy_rows = c.dtype == MOE_DT_BF16 &&
                          (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR || big);
   void* x_perm = copy_rows ? at<void>(ws, L.y_perm) : nullptr;
-  if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
-                           at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks,
-                           err, s) != cudaSuccess)
+  // a small batch without the copy: the whole dispatch in one kernel (the
+  // timer's rank interval; its scan interval stays empty)
+  const bool small = dispatch_small_ok(c, T, x_perm);
+  if (small) {
+    if (launch_dispatch_small(c, T, idx, at<int32_t>(ws, L.counts), offsets, pos, src, err, s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    stage_mark(s);
+    stage_mark(s);
+  } else if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
+                                  at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local),
+                                  L.n_chunks, err, s) != cudaSuccess) {
     return MOE_ERR_CUDA;
+  }
   const DispatchPlace place{&c, T, idx, x, at<int32_t>(ws, L.chunk_hist),
                             at<int32_t>(ws, L.pos_local), pos, src, x_perm};
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
   st = run_experts(c, T, x_perm, src, offsets, w1, w3, w2, x, ws1, ws3, ws2,
                    at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
-                   at<void>(ws, L.row_maps), err, s, &place);
+                   at<void>(ws, L.row_maps), err, s, small ? nullptr : &place, true);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
 }
@@ -450,17 +468,27 @@ moe_status moe_forward_ep(const moe_config* cfg, int64_t T, int32_t expert_begin
   // gathered rows or a permuted copy, by the same rule as moe_forward
   const bool big = T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed;
   void* x_perm = (c.dtype == MOE_DT_BF16 && big) ? at<void>(ws, L.y_perm) : nullptr;
-  if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
-                           at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks,
-                           err, s) != cudaSuccess)
+  // a small batch without the copy: the whole dispatch in one kernel (the
+  // timer's rank interval; its scan interval stays empty)
+  const bool small = dispatch_small_ok(c, T, x_perm);
+  if (small) {
+    if (launch_dispatch_small(c, T, idx, at<int32_t>(ws, L.counts), offsets, pos, src, err, s) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    stage_mark(s);
+    stage_mark(s);
+  } else if (launch_dispatch_sort(c, T, idx, at<int32_t>(ws, L.counts), offsets,
+                                  at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local),
+                                  L.n_chunks, err, s) != cudaSuccess) {
     return MOE_ERR_CUDA;
+  }
   const DispatchPlace place{&c, T, idx, x, at<int32_t>(ws, L.chunk_hist),
                             at<int32_t>(ws, L.pos_local), pos, src, x_perm};
   const int32_t* off_local = offsets + expert_begin;
   void* sbuf = shared_local > 0 ? at<void>(ws, L.s) : nullptr;
   st = run_experts(lc, T, x_perm, src, off_local, w1, w3, w2, x, ws1, ws3, ws2,
                    at<void>(ws, L.y_perm), sbuf, at<void>(ws, L.h), at<void>(ws, L.hs),
-                   at<void>(ws, L.row_maps), err, s, &place);
+                   at<void>(ws, L.row_maps), err, s, small ? nullptr : &place, true);
   if (st != MOE_OK) return st;
   return cuda_status(launch_combine_partial(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf,
                                             off_local, lc.n_routed, y_partial, s));
@@ -590,12 +618,19 @@ const char* moe_status_string(moe_status st) {
 
 int32_t moe_forward_launch_count(const moe_config* cfg, int64_t T) {
   if (check_config(cfg, T) != MOE_OK) return -1;
-  // router: logits + select; dispatch: rank + scan + positions; experts: up
-  // + down, with one kernel that writes the per-expert A maps when the
-  // one-CTA tensor-core kernel runs; combine
-  const bool row_maps = cfg->dtype == MOE_DT_BF16 && (g_expert_kernel == MOE_EXPERT_KERNEL_AUTO ||
-                                                      g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05);
-  return 2 + 3 + 2 + (row_maps ? 1 : 0) + 1;
+  // router: logits + select; dispatch: rank + scan + positions, or one kernel
+  // for a small batch without the row copy (the rule of moe_forward);
+  // experts: up + down, with one kernel that writes the per-expert A maps
+  // when the one-CTA tensor-core kernel runs; combine
+  const moe_config& c = *cfg;
+  const bool row_maps = c.dtype == MOE_DT_BF16 && (g_expert_kernel == MOE_EXPERT_KERNEL_AUTO ||
+                                                   g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05);
+  const bool copy_rows = c.dtype == MOE_DT_BF16 &&
+                         (g_expert_kernel == MOE_EXPERT_KERNEL_TCGEN05_PAIR ||
+                          T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed);
+  const bool small = T * (int64_t)c.topk <= kDispatchSmallPairs &&
+                     c.n_routed <= kDispatchSmallExperts && !copy_rows;
+  return 2 + (small ? 1 : 3) + 2 + (row_maps ? 1 : 0) + 1;
 }
 
 moe_status moe_gate_noalloc(const moe_config* cfg, int64_t T, const void* x, const void* w_router,

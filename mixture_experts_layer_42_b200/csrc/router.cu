@@ -178,6 +178,11 @@ template <int VPL>
 __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a) {
   extern __shared__ float z_s[];  // [8][E] logits of this CTA's tokens
   __shared__ float gsc_s[8][64];
+  // launched as a programmatic dependent of the logits kernel: the dispatch
+  // after it may start; the logits (and the error word) are read after the
+  // logits grid completes
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (a.hold_on_timeout && (*a.hold_on_timeout & ERRBIT_TIMEOUT)) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int E = a.E;
@@ -398,13 +403,15 @@ cudaError_t launch_router(const moe_config& c, int64_t T, const void* x, const v
   unsigned blocks = (unsigned)ceil_div<int64_t>(T, 8);
   int vpl = ceil_div(E, 32);
   const size_t zs = (size_t)8 * E * sizeof(float);
-  if (vpl <= 1) router_select_kernel<1><<<blocks, 256, zs, st>>>(a);
-  else if (vpl <= 2) router_select_kernel<2><<<blocks, 256, zs, st>>>(a);
-  else if (vpl <= 4) router_select_kernel<4><<<blocks, 256, zs, st>>>(a);
-  else if (vpl <= 8) router_select_kernel<8><<<blocks, 256, zs, st>>>(a);
-  else if (vpl <= 16) router_select_kernel<16><<<blocks, 256, zs, st>>>(a);
-  else router_select_kernel<32><<<blocks, 256, zs, st>>>(a);
+  void (*k)(const SelectArgs) = vpl <= 1    ? router_select_kernel<1>
+                                : vpl <= 2  ? router_select_kernel<2>
+                                : vpl <= 4  ? router_select_kernel<4>
+                                : vpl <= 8  ? router_select_kernel<8>
+                                : vpl <= 16 ? router_select_kernel<16>
+                                            : router_select_kernel<32>;
+  err = launch_pdl(pdl_ok(), k, dim3(blocks), dim3(256), zs, st, a);
   stage_mark(st);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

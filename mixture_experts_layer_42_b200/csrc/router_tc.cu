@@ -76,6 +76,9 @@ struct RouterTcArgs {
 };
 
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterTcArgs g) {
+  // the selection, a programmatic dependent of this kernel, may launch now
+  // (it waits for this grid before it reads the logits)
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t* full = reinterpret_cast<uint64_t*>(tiles + RSTAGES * RSTAGE);

@@ -123,9 +123,12 @@ def test_stall_hook_validates_its_argument(M):
 
 def test_launch_count(M):
     # bf16 on the one-CTA tensor-core kernel: the expert GEMMs follow one
-    # kernel that writes their per-expert A maps
-    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 9
-    assert M.moe_forward_launch_count(inputs.CONFIGS["tiny_fp32"], 64) == 8
+    # kernel that writes their per-expert A maps; a small batch that reads
+    # its rows from x is dispatched by one kernel instead of three
+    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 7
+    assert M.moe_forward_launch_count(inputs.CONFIGS["v3_prefill"], 8192) == 9
+    assert M.moe_forward_launch_count(inputs.CONFIGS["tiny_fp32"], 64) == 6
+    assert M.moe_forward_launch_count(inputs.CONFIGS["tiny_fp32"], 4096) == 8
     M.moe_select_expert_kernel(M.MOE_EXPERT_KERNEL_TCGEN05_PAIR)
     try:
         assert M.moe_forward_launch_count(inputs.CONFIGS["v3_decode"], 128) == 8

@@ -169,6 +169,36 @@ def test_dispatch_matches_oracle(name, T, copy_rows):
     _dispatch_check(L, r["idx"], out)
 
 
+@pytest.mark.parametrize("T,E,k,bad", [(1, 8, 2, False), (128, 256, 8, False), (512, 512, 8, False),
+                                       (4096, 16, 1, False), (300, 64, 6, True)])
+def test_one_kernel_dispatch_equals_the_chunked_dispatch(T, E, k, bad):
+    # small batches without the row copy take one kernel (one CTA): the same
+    # counts, offsets, pos and src, bit for bit, as the chunked three-kernel
+    # path that the copy takes (the largest case is exactly 4096 pairs)
+    cfg = bf16_small(T=T, n_routed=E, n_groups=1, topk_groups=1, topk=k, dim=128, n_shared=0)
+    g = torch.Generator().manual_seed(T + E)
+    idx = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(T)]).to(torch.int32)
+    if bad:
+        idx[7, 2] = E + 3            # out of range: flagged, its pair dropped
+        idx[11, 0] = -1
+    idx = idx.cuda()
+    x = torch.randn(T, cfg.dim, generator=g).to(torch.bfloat16).cuda()
+    outs = []
+    for copy in (True, False):
+        ws = M.alloc_workspace(cfg, T)
+        o = [torch.full((n,), -7, dtype=torch.int32, device="cuda") for n in (E, E + 1, T * k, T * k)]
+        xp = torch.empty(T * k, cfg.dim, dtype=torch.bfloat16, device="cuda") if copy else None
+        M.moe_dispatch(cfg, idx, x if copy else None, *o, xp, ws)
+        status = M.moe_check_error(ws)
+        assert status == (M.MOE_ERR_DEVICE_CHECK if bad else M.MOE_OK)
+        outs.append(o)
+    n_valid = int(outs[0][1][E].item())
+    for a, b, name in zip(outs[0], outs[1], ("counts", "offsets", "src", "pos")):
+        if name == "src":            # rows past the valid pairs are not written
+            a, b = a[:n_valid], b[:n_valid]
+        assert torch.equal(a, b), name
+
+
 def test_dispatch_all_tokens_same_experts():
     # extreme skew: every token picks experts {3, 7, 9, 12}
     cfg = bf16_small(T=1000)
