@@ -18,6 +18,9 @@ combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ pos,
                T* __restrict__ y) {
   __shared__ int32_t p_s[32];
   __shared__ float w_s[32];
+  // a programmatic dependent of the down-projection: its outputs are read
+  // after that grid completes
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
     p_s[threadIdx.x] = pos[t * k + threadIdx.x];
@@ -79,6 +82,7 @@ combine_partial_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__
                        float* __restrict__ y) {
   __shared__ int32_t p_s[32];
   __shared__ float w_s[32];
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // as combine_kernel
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
     const int lo = offsets_local[0], hi = offsets_local[n_local];
@@ -146,14 +150,12 @@ cudaError_t launch_combine_partial(const moe_config& c, int64_t T, const void* y
   const int nvec = D * act_bytes(c) / 16;
   dim3 grid((unsigned)T, (unsigned)ceil_div(nvec, 256));
   if (c.dtype == MOE_DT_BF16)
-    combine_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)y_perm, pos, weights, (const __nv_bfloat16*)s, offsets_local, n_local,
-        k, D, y32);
-  else
-    combine_partial_kernel<float><<<grid, 256, 0, st>>>((const float*)y_perm, pos, weights,
-                                                        (const float*)s, offsets_local, n_local, k,
-                                                        D, y32);
-  return cudaGetLastError();
+    return launch_pdl(pdl_ok(), combine_partial_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                      (const __nv_bfloat16*)y_perm, pos, weights, (const __nv_bfloat16*)s,
+                      offsets_local, n_local, k, D, y32);
+  return launch_pdl(pdl_ok(), combine_partial_kernel<float>, grid, dim3(256), 0, st,
+                    (const float*)y_perm, pos, weights, (const float*)s, offsets_local, n_local, k,
+                    D, y32);
 }
 
 cudaError_t launch_cast(const moe_config& c, int64_t T, const float* y32, void* y, cudaStream_t st) {
@@ -172,14 +174,16 @@ cudaError_t launch_combine(const moe_config& c, int64_t T, const void* y_perm, c
   const int D = c.dim, k = c.topk;
   const int nvec = D * act_bytes(c) / 16;
   dim3 grid((unsigned)T, (unsigned)ceil_div(nvec, 256));
+  cudaError_t e;
   if (c.dtype == MOE_DT_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)y_perm, pos, weights, (const __nv_bfloat16*)s, k, D, (__nv_bfloat16*)y);
+    e = launch_pdl(pdl_ok(), combine_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                   (const __nv_bfloat16*)y_perm, pos, weights, (const __nv_bfloat16*)s, k, D,
+                   (__nv_bfloat16*)y);
   else
-    combine_kernel<float><<<grid, 256, 0, st>>>((const float*)y_perm, pos, weights, (const float*)s,
-                                                k, D, (float*)y);
+    e = launch_pdl(pdl_ok(), combine_kernel<float>, grid, dim3(256), 0, st, (const float*)y_perm,
+                   pos, weights, (const float*)s, k, D, (float*)y);
   stage_mark(st);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

@@ -314,13 +314,17 @@ struct Fp8Weights {
 };
 // Activation rows [R, K] (act) to e4m3 with one scale per 1 x 128 block;
 // the scales' row stride is sstride floats (<= 0: K/128).
+// With pos (T * k row positions) and scale_perm, each block's scale is also
+// written to its row's permuted rows (the up-projection's routed row order).
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
-                              float* scale, int sstride, cudaStream_t st);
+                              float* scale, int sstride, cudaStream_t st,
+                              const int32_t* pos = nullptr, float* scale_perm = nullptr);
 // A matrix [R, C] (bf16 or fp32) to e4m3 with one scale per 128 x 128 block.
 cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
                                 float* scale, cudaStream_t st);
 // The FP8 expert GEMMs (gemm_fp8.cu): UP from the quantized x (routed rows
-// through src) into the quantized h, DOWN from it into y_perm and s (act).
+// through src, their scales already in expert order in xs_perm) into the
+// quantized h, DOWN from it into y_perm and s (act).
 cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights& w,
                                const uint8_t* xq, const float* xs, float* xs_perm,
                                const int32_t* src, const int32_t* offsets, uint8_t* hq, float* hsc,

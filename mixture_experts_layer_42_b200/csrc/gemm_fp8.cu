@@ -152,8 +152,9 @@ struct Fp8Args {
   const float* ws1[2];   // weight scales [E, N/128, K/128] of tmW1
   const float* ws3[2];   // of tmW3
   // scales of the A rows [rows, K/128], in the A rows' order: routed UP the
-  // quantized x's scales permuted into expert order (gather_scales_kernel),
-  // so that a tile's are one contiguous run the producer copies in bulk
+  // quantized x's scales in expert order (quant_rows_kernel writes them
+  // through pos), so that a tile's are one contiguous run the producer copies
+  // in bulk
   const float* asc[2];
   const int32_t* src;    // routed UP: the token of each expert-order row
   int a_rows[2];         // rows of the A tensors (an out-of-range row reads zeros)
@@ -235,6 +236,9 @@ __device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)
 
 template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {
+  // the kernel after this one (the combine, after the down-projection) may
+  // launch now; it waits for this grid before it reads the outputs
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int FSTAGES = Ring<UP>::STAGES;
@@ -269,6 +273,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    // a programmatic dependent (up-projection): wait for the kernel before it
+    // before anything it or its predecessors wrote is read (the offsets here;
+    // src, the scales and x's codes after the __syncthreads below)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // token chunks per expert and their exclusive prefix
     const int per = (E + 31) / 32;
     int lsum = 0;
@@ -604,10 +612,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
 
 // Rows [R, K] (act) to e4m3 with one power-of-two scale per 1 x 128 block:
 // one warp per block, 4 elements per lane.
+// With pos, each block's scale is also written to the k permuted rows of its
+// row's (token, slot) pairs (scale_perm, for the up-projection's routed rows;
+// pairs with pos < 0 are skipped).
 template <typename T>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int64_t R, int K,
                                                          uint8_t* __restrict__ q,
-                                                         float* __restrict__ scale, int sstride) {
+                                                         float* __restrict__ scale, int sstride,
+                                                         const int32_t* __restrict__ pos, int k,
+                                                         float* __restrict__ scale_perm) {
+  // a programmatic dependent of the dispatch (pos): the up-projection after
+  // it may launch now; pos is read after the dispatch's grid completes
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int kbn = K / QB;
   const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
@@ -626,21 +643,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
 #pragma unroll
   for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(ldexpf(v[i], -se)) << (8 * i);
   reinterpret_cast<uint32_t*>(q + r * K + kb * QB)[lane] = packed;
-  if (lane == 0) scale[r * sstride + kb] = ldexpf(1.f, se);
-}
-
-// The quantized x's scales in expert order: row p takes token src[p]'s
-// (rows at or past offsets[E] are not read by the experts and are skipped).
-__global__ void __launch_bounds__(256) gather_scales_kernel(const float* __restrict__ xs,
-                                                            const int32_t* __restrict__ src,
-                                                            const int32_t* __restrict__ offsets,
-                                                            int E, int64_t Tk, int sstride,
-                                                            float* __restrict__ xs_perm) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t p = i / sstride;
-  const int kb = (int)(i % sstride);
-  if (p >= Tk || p >= offsets[E]) return;
-  xs_perm[i] = xs[(int64_t)src[p] * sstride + kb];
+  const float sc = ldexpf(1.f, se);
+  if (lane == 0) scale[r * sstride + kb] = sc;
+  if (pos != nullptr && lane < k) {
+    const int p = pos[r * k + lane];
+    if (p >= 0) scale_perm[(int64_t)p * sstride + kb] = sc;
+  }
 }
 
 // A bf16 / fp32 matrix [R, C] to e4m3 with one power-of-two scale per
@@ -715,17 +723,17 @@ bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uin
 }  // namespace
 
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
-                              float* scale, int sstride, cudaStream_t st) {
+                              float* scale, int sstride, cudaStream_t st, const int32_t* pos,
+                              float* scale_perm) {
   const int64_t warps = R * (K / QB);
   if (warps == 0) return cudaSuccess;
   if (sstride <= 0) sstride = K / QB;
   const unsigned blocks = (unsigned)ceil_div<int64_t>(warps * 32, 256);
   if (c.dtype == MOE_DT_BF16)
-    quant_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)a, R, K, q, scale,
-                                                              sstride);
-  else
-    quant_rows_kernel<float><<<blocks, 256, 0, st>>>((const float*)a, R, K, q, scale, sstride);
-  return cudaGetLastError();
+    return launch_pdl(pdl_ok(), quant_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                      (const __nv_bfloat16*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm);
+  return launch_pdl(pdl_ok(), quant_rows_kernel<float>, dim3(blocks), dim3(256), 0, st,
+                    (const float*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm);
 }
 
 int fp8_scale_stride(int K) { return scale_stride(K); }
@@ -752,12 +760,6 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
   const int64_t Tk = T * c.topk;
   const bool sh = Is > 0;
   cudaError_t e;
-  {
-    const int ss = scale_stride(D);
-    gather_scales_kernel<<<(unsigned)ceil_div<int64_t>(Tk * ss, 256), 256, 0, st>>>(
-        xs, src, offsets, E, Tk, ss, xs_perm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
   for (int pass = 0; pass < 2; ++pass) {
     const bool up = pass == 0;
     Fp8Args g;
@@ -840,7 +842,9 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
         e = cudaFuncSetAttribute(grouped_fp8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)FSMEM);
         if (e != cudaSuccess) return e;
-        grouped_fp8_kernel<true><<<grid, NTHREADS, FSMEM, st>>>(g);
+        // a programmatic dependent of the row quantization (or the scale gather)
+        e = launch_pdl(pdl_ok(), grouped_fp8_kernel<true>, dim3(grid), dim3(NTHREADS), FSMEM, st, g);
+        if (e != cudaSuccess) return e;
       } else {
         e = cudaFuncSetAttribute(grouped_fp8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)FSMEM);

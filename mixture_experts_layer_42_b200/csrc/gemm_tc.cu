@@ -151,6 +151,9 @@ __device__ __forceinline__ float silu_fast(float u) { return u / (1.0f + __expf(
 
 template <bool UP>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid_constant__ TcArgs g) {
+  // the kernel after this one (the combine, after the down-projection) may
+  // launch now; it waits for this grid before it reads the outputs
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* tiles = base;

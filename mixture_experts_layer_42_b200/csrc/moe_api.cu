@@ -569,10 +569,12 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
                       at<int32_t>(ws, L.chunk_hist), at<int32_t>(ws, L.pos_local), L.n_chunks, err,
                       s) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // x to e4m3 once per step (its kernel is timed with the up-projection)
+  // x to e4m3 once per step, each block's scale also to the routed pairs'
+  // permuted rows (its kernel is timed with the up-projection)
   uint8_t* xq = at<uint8_t>(ws, F.xq);
   float* xs = at<float>(ws, F.xs);
-  if (launch_quant_rows(c, x, T, c.dim, xq, xs, fp8_stride_host(c.dim), s) != cudaSuccess)
+  if (launch_quant_rows(c, x, T, c.dim, xq, xs, fp8_stride_host(c.dim), s, pos,
+                        at<float>(ws, F.xs_perm)) != cudaSuccess)
     return MOE_ERR_CUDA;
   Fp8Weights fw{static_cast<const uint8_t*>(w->w1), static_cast<const uint8_t*>(w->w3),
                 static_cast<const uint8_t*>(w->w2), static_cast<const uint8_t*>(w->ws1),
