@@ -263,9 +263,8 @@ cudaError_t launch_router_logits_tc(const moe_config& c, int64_t T, const void* 
 size_t gate_scratch_floats();
 cudaError_t gate_scratch_current_device(float** scratch, uint32_t** err);
 
-// x_perm may be null: then only counts, offsets, src and pos are written.
-// zero_ctr (nullable): an int the scan kernel sets to 0 (the up-projection's
-// tile counter, when the experts follow in the same stream).
+// x_perm may be null: then only counts, offsets, src and pos are written (by
+// one kernel for a small batch, dispatch_small_ok).
 cudaError_t launch_dispatch(const moe_config& c, int64_t T, const int32_t* idx, const void* x,
                             int32_t* counts, int32_t* offsets, int32_t* src, int32_t* pos,
                             void* x_perm, int32_t* chunk_hist, int32_t* pos_local, int n_chunks,

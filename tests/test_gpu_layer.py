@@ -448,6 +448,39 @@ def test_stage_timing_records_one_call_in_every():
     assert n == 4 and ms["router_logits"] > 0
 
 
+@pytest.mark.parametrize("kw", [dict(T=64), dict(T=1500)], ids=["one_kernel_dispatch", "chunked_dispatch"])
+def test_back_to_back_forwards_on_one_stream(kw):
+    # the forward's kernels are chained as programmatic dependent launches:
+    # eight forwards issued back to back on one stream, x rewritten on the
+    # stream between them and no host synchronisation, must each give the
+    # output of that x run alone
+    cfg = bf16_small(**kw)
+    L = Layer(cfg)
+    w1, w3, w2, ws1, ws3, ws2 = L.w
+    gen = torch.Generator().manual_seed(5)
+    xs = [torch.randn(L.T, cfg.dim, generator=gen).to(cfg.torch_dtype).cuda() for _ in range(8)]
+    ws = M.alloc_workspace(cfg, L.T)
+    x = torch.empty_like(L.x)
+    refs = []
+    for xi in xs:
+        x.copy_(xi)
+        y = torch.empty(L.T, cfg.dim, dtype=cfg.torch_dtype, device="cuda")
+        M.moe_forward(cfg, x, L.w_r, L.bias, w1, w3, w2, ws1, ws3, ws2, y, ws)
+        torch.cuda.synchronize()
+        refs.append(y)
+    s = torch.cuda.Stream()
+    ys = [torch.empty_like(r) for r in refs]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        for xi, y in zip(xs, ys):
+            x.copy_(xi)
+            M.moe_forward(cfg, x, L.w_r, L.bias, w1, w3, w2, ws1, ws3, ws2, y, ws, stream=s)
+    torch.cuda.synchronize()
+    assert M.moe_check_error(ws) == M.MOE_OK
+    for y, r in zip(ys, refs):
+        assert torch.equal(y, r)
+
+
 def test_forward_replays_from_a_cuda_graph():
     # moe_forward does no host synchronisation and allocates nothing, so it can
     # be captured once and replayed with new inputs written into the same buffers
