@@ -154,3 +154,27 @@ def test_fp8_shapes_are_checked():
     with pytest.raises(M.MoEError) as e:
         M.moe_workspace_size_fp8(inputs.CONFIGS["tiny_fp32"], 64)
     assert e.value.status == M.MOE_ERR_UNSUPPORTED
+
+
+def test_fp8_forward_with_zero_and_tiny_rows():
+    # a token row of zeros (its blocks' scale 2^0, UE8M0 byte 127) and rows so
+    # small that their blocks take the smallest scale, 2^-127 (UE8M0 byte 0),
+    # through the block-scaled forward, against the oracle's FP8 layer
+    cfg = small(T=64)
+    L = Layer(cfg)
+    x = L.x.float()
+    x[0] = 0.0
+    x[1:4] = x[1:4] * 2.0 ** -125
+    L.x = x.to(torch.bfloat16).contiguous()
+    xq, xs = quantize(cfg, L.x, 1)
+    s = xs.cpu().numpy()
+    assert (s[0] == 1.0).all() and (s[1:4] == 2.0 ** -127).mean() > 0.5
+    F = Fp8Layer(L)
+    y, wts, idx = F.forward()
+    r = L.oracle_route()
+    differs = check_routing(cfg, idx, wts, r)
+    rows = np.nonzero(~differs)[0]
+    assert {0, 1, 2, 3} <= set(rows.tolist())
+    yref = O.moe_layer(host(L.x), r["weights"], r["idx"], F.experts(), F.shared(), act_dtype="bf16",
+                       tokens=rows, fp8=True)
+    assert check_y(cfg, to_np(y)[rows], yref) < 2e-2
