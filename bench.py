@@ -77,6 +77,8 @@ def parse(argv=None):
                     help="override the number of routed experts (smaller cases for profiling)")
     ap.add_argument("--expert-kernel", default="auto", choices=["auto", "simt", "one_cta", "pair"],
                     help="GEMM kernels of a bf16 layer (moe_select_expert_kernel)")
+    ap.add_argument("--fp8-kernel", default="auto", choices=["auto", "tokens_on_n", "tokens_on_m"],
+                    help="form of the FP8 expert GEMMs (moe_select_fp8_kernel)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other workloads' measurements (N=1 only runs them)")
     ap.add_argument("--routing-only", action="store_true",
@@ -568,6 +570,8 @@ def ours_arm(a, D):
     M.moe_select_expert_kernel({"auto": M.MOE_EXPERT_KERNEL_AUTO, "simt": M.MOE_EXPERT_KERNEL_SIMT,
                                 "one_cta": M.MOE_EXPERT_KERNEL_TCGEN05,
                                 "pair": M.MOE_EXPERT_KERNEL_TCGEN05_PAIR}[a.expert_kernel])
+    M.moe_select_fp8_kernel({"auto": M.MOE_FP8_KERNEL_AUTO, "tokens_on_n": M.MOE_FP8_KERNEL_TOKENS_ON_N,
+                             "tokens_on_m": M.MOE_FP8_KERNEL_TOKENS_ON_M}[a.fp8_kernel])
     S = Setup(cfg, dev)
     T = cfg.T
     launches = M.moe_forward_launch_count(cfg, T)

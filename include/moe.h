@@ -269,7 +269,13 @@ MOE_API moe_status moe_workspace_size_fp8(const moe_config* cfg, int64_t T, size
  * (w3 x) quantized the same way
  * before w2, each expert's output rounded to bf16, and the combine as in
  * moe_forward. Workspace of moe_workspace_size_fp8() bytes, initialised by
- * moe_workspace_init(). bf16 layers only. */
+ * moe_workspace_init(). bf16 layers only.
+ * Two forms of the expert GEMMs compute the same sums (see
+ * moe_select_fp8_kernel): for batches of at most 64 rows per expert on
+ * average, the weights on the MMA's M side and up to 32 tokens of an expert on
+ * its N side (each weight tile streamed once per 32 tokens); above that, 128
+ * token rows on M and 256 weight rows on N, the routed rows' codes written in
+ * expert order by the row quantization. */
 MOE_API moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x,
                                    const void* w_router, const float* bias,
                                    const moe_fp8_weights* w, void* y, float* weights_out,
@@ -366,6 +372,21 @@ enum {
   MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
 };
 MOE_API moe_status moe_select_expert_kernel(int32_t which);
+
+/* Which form runs the expert GEMMs of moe_forward_fp8, process-wide (for
+ * checks and measurement):
+ *   AUTO (default)  by the batch: tokens on N for at most 64 (token, slot)
+ *                   rows per expert on average, tokens on M above;
+ *   TOKENS_ON_N     weights on the MMA's M side, up to 32 tokens on N;
+ *   TOKENS_ON_M     128 token rows on M, 256 weight rows on N.
+ * Both give the same results up to the order of the fp32 sums. Returns
+ * MOE_ERR_INVALID_ARG for other values. */
+enum {
+  MOE_FP8_KERNEL_AUTO = 0,
+  MOE_FP8_KERNEL_TOKENS_ON_N = 1,
+  MOE_FP8_KERNEL_TOKENS_ON_M = 2
+};
+MOE_API moe_status moe_select_fp8_kernel(int32_t which);
 
 /* Test hook for the failure path of the tensor-core pipelines, process-wide,
  * off by default; the pages have no counterpart. While enabled, one kernel

@@ -32,6 +32,7 @@ MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX = 0, 1
 MOE_EXPERT_KERNEL_AUTO, MOE_EXPERT_KERNEL_SIMT, MOE_EXPERT_KERNEL_TCGEN05 = 0, 1, 2
 MOE_EXPERT_KERNEL_TCGEN05_PAIR = 3
+MOE_FP8_KERNEL_AUTO, MOE_FP8_KERNEL_TOKENS_ON_N, MOE_FP8_KERNEL_TOKENS_ON_M = 0, 1, 2
 MOE_STALL_NONE, MOE_STALL_EXPERTS_UP, MOE_STALL_ROUTER = 0, 1, 2
 
 # Every symbol include/moe.h declares.
@@ -41,7 +42,8 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch
            "moe_stage_timing_begin", "moe_stage_timing_end", "moe_gate_noalloc",
            "moe_stage_timing_begin_every", "moe_debug_stall_pipeline",
            "moe_gate_noalloc_check_error", "moe_experts_grouped_gather", "moe_forward_ep",
-           "moe_cast_output", "moe_quantize_fp8", "moe_workspace_size_fp8", "moe_forward_fp8")
+           "moe_cast_output", "moe_quantize_fp8", "moe_workspace_size_fp8", "moe_forward_fp8",
+           "moe_select_fp8_kernel")
 
 # Kernels of moe_forward, in launch order.
 STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_pos",
@@ -87,6 +89,7 @@ def _load() -> ctypes.CDLL:
         "moe_status_string": [I32],
         "moe_forward_launch_count": [C, I64],
         "moe_select_expert_kernel": [I32],
+        "moe_select_fp8_kernel": [I32],
         "moe_stage_timing_begin": [I32],
         "moe_stage_timing_begin_every": [I32, I32],
         "moe_debug_stall_pipeline": [I32],
@@ -277,6 +280,10 @@ def moe_debug_stall_pipeline(enable: int) -> None:
 
 def moe_select_expert_kernel(which: int) -> None:
     _check(_lib.moe_select_expert_kernel(int(which)), "moe_select_expert_kernel")
+
+
+def moe_select_fp8_kernel(which: int) -> None:
+    _check(_lib.moe_select_fp8_kernel(int(which)), "moe_select_fp8_kernel")
 
 
 def moe_stage_timing_begin(max_calls: int) -> None:

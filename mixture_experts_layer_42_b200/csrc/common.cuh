@@ -71,6 +71,7 @@ constexpr int kFp8Block = 128;
 struct Fp8Layout {
   size_t xq, xs;        // quantized x [T, D] e4m3, its scales [T, D/128] fp32
   size_t xs_perm;       // x's scales in expert order [T*k, D/128]
+  size_t xq_perm;       // x's codes in expert order [T*k, D] (token-on-M form)
   size_t hq, hs;        // quantized h [T*k, I], scales [T*k, I/128]
   size_t hsq, hss;      // the shared MLP's h [T, I_s], scales [T, I_s/128]
   size_t total;
@@ -108,6 +109,7 @@ inline Fp8Layout fp8_layout(const moe_config& c, int64_t T, size_t base) {
   L.xq = take((size_t)T * D);
   L.xs = take((size_t)T * fp8_stride_host((int)D) * 4);
   L.xs_perm = take((size_t)T * k * fp8_stride_host((int)D) * 4);
+  L.xq_perm = take((size_t)T * k * D);
   L.hq = take((size_t)T * k * I);
   L.hs = take((size_t)T * k * fp8_stride_host((int)I) * 4);
   L.hsq = take((size_t)T * (Is > 0 ? Is : 1));
@@ -314,10 +316,12 @@ struct Fp8Weights {
 // Activation rows [R, K] (act) to e4m3 with one scale per 1 x 128 block;
 // the scales' row stride is sstride floats (<= 0: K/128).
 // With pos (T * k row positions) and scale_perm, each block's scale is also
-// written to its row's permuted rows (the up-projection's routed row order).
+// written to its row's permuted rows (the up-projection's routed row order),
+// and with q_perm ([T * k, K]) its codes too.
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
                               float* scale, int sstride, cudaStream_t st,
-                              const int32_t* pos = nullptr, float* scale_perm = nullptr);
+                              const int32_t* pos = nullptr, float* scale_perm = nullptr,
+                              uint8_t* q_perm = nullptr);
 // A matrix [R, C] (bf16 or fp32) to e4m3 with one scale per 128 x 128 block.
 cudaError_t launch_quant_blocks(bool bf16, const void* a, int64_t R, int C, uint8_t* q,
                                 float* scale, cudaStream_t st);
@@ -329,6 +333,14 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
                                const int32_t* src, const int32_t* offsets, uint8_t* hq, float* hsc,
                                uint8_t* hsq, float* hss, void* y_perm, void* s, uint32_t* err,
                                int num_sms, cudaStream_t st);
+// The same GEMMs with 128 token rows on the MMA's M side (gemm_fp8m.cu), for
+// batches with many rows per expert: UP reads the routed rows' codes in
+// expert order from xq_perm (scales xs_perm) and the shared MLP's from xq.
+cudaError_t launch_grouped_fp8m(const moe_config& c, int64_t T, const Fp8Weights& w,
+                                const uint8_t* xq, const float* xs, const uint8_t* xq_perm,
+                                const float* xs_perm, const int32_t* offsets, uint8_t* hq,
+                                float* hsc, uint8_t* hsq, float* hss, void* y_perm, void* s,
+                                uint32_t* err, int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
 // Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).

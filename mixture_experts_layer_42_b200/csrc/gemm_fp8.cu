@@ -29,17 +29,15 @@
 // tile::gather4 from the routed rows' tokens or the rows themselves; rows
 // past a tile's tokens read zeros), warp 1 MMA, warps 2-5 epilogue. Waits are
 // bounded as in the bf16 kernel (1 s, then the abort path).
-#include "tc_common.cuh"
-
-#include <cuda_fp8.h>
+#include "fp8_common.cuh"
 
 namespace moe {
 
 namespace {
 
 using namespace tc;
+using namespace fp8;
 
-constexpr int QB = 128;                        // scale block edge; K per stage; weight rows per tile
 constexpr int NT = 32;                         // tokens per tile at most (MMA N)
 constexpr int A_BYTES = NT * QB;               // 4 KB of token rows
 constexpr int W_BYTES = QB * QB;               // 16 KB per weight tile
@@ -96,48 +94,6 @@ constexpr int SC_SLOT = NT * MAX_KB * 4;      // one tile's token scales (8 KB)
 constexpr size_t FSMEM = 1024 + (size_t)RING_BYTES + 9 * 2 * SF_BYTES + 512 +
                          2 * (MAXE + 1) * 4 + 16 + 2 * (size_t)SC_SLOT + 4 * NT * 4;
 static_assert(5 * 3 * SF_BYTES <= 9 * 2 * SF_BYTES, "UP scale-factor bytes");
-
-// kind::mxf8f6f4 block-scaled instruction descriptor: e4m3 A and B, both
-// K-major, fp32 accumulator, UE8M0 scale factors (bit 23), byte `sf` of A's
-// and B's TMEM scale words (bits 29-30 and 4-5), M x N.
-__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t sf) {
-  return (sf << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
-         (sf << 29);
-}
-
-// D[M x N] (+)= (A * 2^SFA) (B * 2^SFB)^T over K = 32: one UE8M0 scale per row
-// of A and per row of B (tcgen05 block scaling, one scale vector per 32 K).
-__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
-      : "memory");
-}
-
-// Shared-memory descriptor of a 32 x 16-byte matrix, no swizzle, rows 16
-// bytes apart (8-row core matrices 128 bytes apart): the source of a
-// tcgen05.cp 32x128b.
-__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)(128 >> 4) << 16) |
-         ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
-}
-
-// TMEM lanes 32w + r (w = 0..3) <- shared row r (16 bytes), r = 0..31.
-__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
-
-// The UE8M0 byte of a power-of-two scale 2^s, -127 <= s <= 127: the biased
-// exponent field of its fp32 encoding (2^-127 is the subnormal with a zero
-// exponent field, which is UE8M0's code 0).
-__device__ __forceinline__ uint32_t ue8m0(float scale) {
-  return (__float_as_uint(scale) >> 23) & 0xFFu;
-}
 
 struct Fp8Args {
   // token rows (uint8 [rows, K], box 128 x 1, for tile::gather4): [0] routed
@@ -207,31 +163,6 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i, int& hint) {
   }
   return t;
 }
-
-// Row stride, in floats, of the activation scales inside the layer: K/128
-// rounded up to a multiple of 4, so every row starts 16-byte aligned and a
-// tile's rows can be copied in one bulk copy.
-__host__ __device__ __forceinline__ int scale_stride(int K) { return ((K / QB) + 3) & ~3; }
-
-// Smallest s with amax <= 448 * 2^s (0 for amax == 0), and at least -127,
-// the smallest scale UE8M0 encodes (blocks whose largest magnitude is below
-// 448 * 2^-127 keep that scale): amax = m 2^e with 0.5 <= m < 1, so s = e - 9,
-// plus one when 2m > 1.75.
-__device__ __forceinline__ int block_exp(float amax) {
-  if (!(amax > 0.f)) return 0;
-  int e;
-  const float m = frexpf(amax, &e);
-  const int s = e - 9 + (2.f * m > 1.75f ? 1 : 0);
-  return s < -127 ? -127 : s;
-}
-
-// (Values are brought into range with ldexpf(v, -s): the reciprocal 2^-s of
-// a tiny block's scale would overflow fp32, the scaled value does not.)
-__device__ __forceinline__ uint8_t to_e4m3(float v) {
-  return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
-}
-
-__device__ __forceinline__ float silu_f(float u) { return u / (1.0f + __expf(-u)); }
 
 
 template <bool UP>
@@ -614,13 +545,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
 // one warp per block, 4 elements per lane.
 // With pos, each block's scale is also written to the k permuted rows of its
 // row's (token, slot) pairs (scale_perm, for the up-projection's routed rows;
-// pairs with pos < 0 are skipped).
+// pairs with pos < 0 are skipped), and with q_perm its codes too (the
+// token-on-M up-projection reads its routed rows from there).
 template <typename T>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a, int64_t R, int K,
                                                          uint8_t* __restrict__ q,
                                                          float* __restrict__ scale, int sstride,
                                                          const int32_t* __restrict__ pos, int k,
-                                                         float* __restrict__ scale_perm) {
+                                                         float* __restrict__ scale_perm,
+                                                         uint8_t* __restrict__ q_perm) {
   // a programmatic dependent of the dispatch (pos): the up-projection after
   // it may launch now; pos is read after the dispatch's grid completes
   asm volatile("griddepcontrol.launch_dependents;");
@@ -645,9 +578,15 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
   reinterpret_cast<uint32_t*>(q + r * K + kb * QB)[lane] = packed;
   const float sc = ldexpf(1.f, se);
   if (lane == 0) scale[r * sstride + kb] = sc;
-  if (pos != nullptr && lane < k) {
-    const int p = pos[r * k + lane];
+  if (pos != nullptr) {
+    const int p = lane < k ? pos[r * k + lane] : -1;
     if (p >= 0) scale_perm[(int64_t)p * sstride + kb] = sc;
+    if (q_perm != nullptr) {
+      for (int j = 0; j < k; ++j) {   // k <= 32
+        const int pj = __shfl_sync(0xffffffffu, p, j);
+        if (pj >= 0) reinterpret_cast<uint32_t*>(q_perm + (int64_t)pj * K + kb * QB)[lane] = packed;
+      }
+    }
   }
 }
 
@@ -683,6 +622,10 @@ __global__ void __launch_bounds__(256) quant_blocks_kernel(const T* __restrict__
   }
   if (threadIdx.x == 0) scale[br * nbc + bc] = ldexpf(1.f, se);
 }
+
+}  // namespace
+
+namespace fp8 {
 
 bool map_u8_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t K) {
   auto fn = encode_fn();
@@ -720,20 +663,20 @@ bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
+}  // namespace fp8
 
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
                               float* scale, int sstride, cudaStream_t st, const int32_t* pos,
-                              float* scale_perm) {
+                              float* scale_perm, uint8_t* q_perm) {
   const int64_t warps = R * (K / QB);
   if (warps == 0) return cudaSuccess;
   if (sstride <= 0) sstride = K / QB;
   const unsigned blocks = (unsigned)ceil_div<int64_t>(warps * 32, 256);
   if (c.dtype == MOE_DT_BF16)
     return launch_pdl(pdl_ok(), quant_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
-                      (const __nv_bfloat16*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm);
+                      (const __nv_bfloat16*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm, q_perm);
   return launch_pdl(pdl_ok(), quant_rows_kernel<float>, dim3(blocks), dim3(256), 0, st,
-                    (const float*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm);
+                    (const float*)a, R, K, q, scale, sstride, pos, c.topk, scale_perm, q_perm);
 }
 
 int fp8_scale_stride(int K) { return scale_stride(K); }

@@ -12,6 +12,8 @@ namespace {
 
 // Which kernel runs the expert GEMMs of a bf16 layer (see moe_select_expert_kernel).
 int g_expert_kernel = MOE_EXPERT_KERNEL_AUTO;
+// Which form runs the FP8 expert GEMMs (see moe_select_fp8_kernel).
+int g_fp8_kernel = MOE_FP8_KERNEL_AUTO;
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -212,6 +214,10 @@ struct TimedCall {
 // rows from x instead of copying them (the swapped-tile limit of the one-CTA
 // tensor-core kernel).
 constexpr int64_t kGatherRows = 64;
+
+// Average rows per expert above which moe_forward_fp8 runs its expert GEMMs
+// with the tokens on the MMA's M side.
+constexpr int64_t kFp8TokensOnMRows = 64;
 
 bool fp8_shapes_ok(const moe_config& c) {
   const int B = kFp8Block;
@@ -570,11 +576,16 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
                       s) != cudaSuccess)
     return MOE_ERR_CUDA;
   // x to e4m3 once per step, each block's scale also to the routed pairs'
-  // permuted rows (its kernel is timed with the up-projection)
+  // permuted rows, and for the token-on-M form their codes too (its kernel
+  // is timed with the up-projection)
+  const bool on_m = g_fp8_kernel == MOE_FP8_KERNEL_TOKENS_ON_M ||
+                    (g_fp8_kernel == MOE_FP8_KERNEL_AUTO &&
+                     T * (int64_t)c.topk > kFp8TokensOnMRows * c.n_routed);
   uint8_t* xq = at<uint8_t>(ws, F.xq);
   float* xs = at<float>(ws, F.xs);
+  uint8_t* xq_perm = on_m ? at<uint8_t>(ws, F.xq_perm) : nullptr;
   if (launch_quant_rows(c, x, T, c.dim, xq, xs, fp8_stride_host(c.dim), s, pos,
-                        at<float>(ws, F.xs_perm)) != cudaSuccess)
+                        at<float>(ws, F.xs_perm), xq_perm) != cudaSuccess)
     return MOE_ERR_CUDA;
   Fp8Weights fw{static_cast<const uint8_t*>(w->w1), static_cast<const uint8_t*>(w->w3),
                 static_cast<const uint8_t*>(w->w2), static_cast<const uint8_t*>(w->ws1),
@@ -582,11 +593,16 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
                 w->w1_scale, w->w3_scale, w->w2_scale, w->ws1_scale, w->ws3_scale, w->ws2_scale};
   const bool sh = c.shared_inter > 0;
   void* sbuf = sh ? at<void>(ws, L.s) : nullptr;
-  if (launch_grouped_fp8(c, T, fw, xq, xs, at<float>(ws, F.xs_perm), src, offsets,
-                         at<uint8_t>(ws, F.hq), at<float>(ws, F.hs),
-                         at<uint8_t>(ws, F.hsq), at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf,
-                         err, num_sms_current(), s) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  const cudaError_t ge =
+      on_m ? launch_grouped_fp8m(c, T, fw, xq, xs, xq_perm, at<float>(ws, F.xs_perm), offsets,
+                                 at<uint8_t>(ws, F.hq), at<float>(ws, F.hs), at<uint8_t>(ws, F.hsq),
+                                 at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf, err,
+                                 num_sms_current(), s)
+           : launch_grouped_fp8(c, T, fw, xq, xs, at<float>(ws, F.xs_perm), src, offsets,
+                                at<uint8_t>(ws, F.hq), at<float>(ws, F.hs), at<uint8_t>(ws, F.hsq),
+                                at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf, err,
+                                num_sms_current(), s);
+  if (ge != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_status(launch_combine(c, T, at<void>(ws, L.y_perm), pos, weights, sbuf, y, s));
 }
 
@@ -725,6 +741,14 @@ moe_status moe_select_expert_kernel(int32_t which) {
       which != MOE_EXPERT_KERNEL_TCGEN05 && which != MOE_EXPERT_KERNEL_TCGEN05_PAIR)
     return MOE_ERR_INVALID_ARG;
   g_expert_kernel = which;
+  return MOE_OK;
+}
+
+moe_status moe_select_fp8_kernel(int32_t which) {
+  if (which != MOE_FP8_KERNEL_AUTO && which != MOE_FP8_KERNEL_TOKENS_ON_N &&
+      which != MOE_FP8_KERNEL_TOKENS_ON_M)
+    return MOE_ERR_INVALID_ARG;
+  g_fp8_kernel = which;
   return MOE_OK;
 }
 

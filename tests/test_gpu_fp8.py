@@ -20,6 +20,18 @@ from tests.gpu_util import Layer, check_routing, check_y, host, to_np
 
 pytestmark = pytest.mark.gpu
 
+# The two forms of the FP8 expert GEMMs: weights on the MMA's M side with up
+# to 32 tokens on N (decode batches), and 128 token rows on M with 256 weight
+# rows on N (large batches).
+FORMS = {"tokens_on_n": M.MOE_FP8_KERNEL_TOKENS_ON_N, "tokens_on_m": M.MOE_FP8_KERNEL_TOKENS_ON_M}
+
+
+@pytest.fixture(params=sorted(FORMS))
+def form(request):
+    M.moe_select_fp8_kernel(FORMS[request.param])
+    yield request.param
+    M.moe_select_fp8_kernel(M.MOE_FP8_KERNEL_AUTO)
+
 
 def small(**kw):
     base = inputs.MoEConfig("fp8_small", T=300, dim=384, n_routed=16, n_groups=4, topk_groups=2,
@@ -131,7 +143,20 @@ def _parity(cfg):
                                 dict(n_shared=0), dict(n_routed=64, n_groups=8, topk_groups=3, topk=6),
                                 dict(T=1000, n_routed=8, n_groups=2, topk_groups=1, topk=2),
                                 dict(score="softmax", bias="none", n_groups=1, topk_groups=1, n_shared=2)])
-def test_fp8_forward_matches_oracle(kw):
+def test_fp8_forward_matches_oracle(kw, form):
+    err, *_ = _parity(small(**kw))
+    assert err < 2e-2
+
+
+@pytest.mark.parametrize("kw", [dict(T=2048, n_routed=8, n_groups=2, topk_groups=1, topk=2, dim=512,
+                                     moe_inter=384),
+                                dict(T=700, n_routed=4, n_groups=1, topk_groups=1, topk=1, n_shared=0),
+                                dict(T=513, dim=256, moe_inter=128, n_routed=2, n_groups=1,
+                                     topk_groups=1, topk=2)])
+def test_fp8_forward_many_rows_per_expert(kw, form):
+    # experts with several 128-row tiles and ragged last tiles; a layer with
+    # dim an odd multiple of 128 (its last down-projection tile one weight
+    # block wide) and every expert taking every token
     err, *_ = _parity(small(**kw))
     assert err < 2e-2
 
@@ -156,7 +181,7 @@ def test_fp8_shapes_are_checked():
     assert e.value.status == M.MOE_ERR_UNSUPPORTED
 
 
-def test_fp8_forward_with_zero_and_tiny_rows():
+def test_fp8_forward_with_zero_and_tiny_rows(form):
     # a token row of zeros (its blocks' scale 2^0, UE8M0 byte 127) and rows so
     # small that their blocks take the smallest scale, 2^-127 (UE8M0 byte 0),
     # through the block-scaled forward, against the oracle's FP8 layer
@@ -178,3 +203,27 @@ def test_fp8_forward_with_zero_and_tiny_rows():
     yref = O.moe_layer(host(L.x), r["weights"], r["idx"], F.experts(), F.shared(), act_dtype="bf16",
                        tokens=rows, fp8=True)
     assert check_y(cfg, to_np(y)[rows], yref) < 2e-2
+
+
+@pytest.mark.slow
+def test_fp8_forward_v3_prefill_sampled_tokens():
+    # the DeepSeek-V3 prefill batch (T = 8192) with its weights in the FP8
+    # layout, in the form the layer picks for it (tokens on M): routing on
+    # every token, outputs on a seeded sample that includes tokens of the most
+    # and least loaded experts and the first and last token
+    cfg = inputs.CONFIGS["v3_prefill"]
+    L = Layer(cfg)
+    F = Fp8Layer(L)
+    y, wts, idx = F.forward()
+    r = L.oracle_route()
+    differs = check_routing(cfg, idx, wts, r)
+    rng = np.random.default_rng(11)
+    counts = np.bincount(r["idx"].ravel(), minlength=cfg.n_routed)
+    hot, cold = int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    picks = [np.nonzero((r["idx"] == hot).any(1))[0][:3], np.nonzero((r["idx"] == cold).any(1))[0][:3],
+             [0, L.T - 1], rng.choice(L.T, 40, replace=False)]
+    tokens = np.unique(np.concatenate(picks))
+    tokens = tokens[~differs[tokens]]
+    yref = O.moe_layer(host(L.x), r["weights"], r["idx"], F.experts(), F.shared(), act_dtype="bf16",
+                       tokens=tokens, fp8=True)
+    assert check_y(cfg, to_np(y)[tokens], yref) < 2e-2
