@@ -22,9 +22,9 @@ memory and y copied back every step; the roofline of the dominant kernel from
 per-kernel CUDA events recorded in a separate untimed pass after the timed
 loop (which records no other event); the layer roofline; the CPU oracle's rate on a bounded token sample (N=1
 only); SM clocks sampled during the run. At N=1 the line also carries
-`workloads`: the same device-timed measurements for the other bf16 workloads
-(V3 prefill, the Zipf-skewed prefill, the softmax layer), each timed for about
-a second.
+`workloads`: the same device-timed measurements for the other workloads (V3
+prefill, the Zipf-skewed prefill, the softmax layer, and the V3 decode and
+prefill batches with FP8 expert weights), each timed for about a second.
 
 --impl reference times the CPU oracle (the plain fp64 statement of the layer)
 on the host cores, on the same workload, metric and unit.
@@ -333,6 +333,7 @@ def config_dict(cfg, N, expert_kernel, l2):
             "topk": cfg.topk, "moe_inter": cfg.moe_inter, "shared_inter": cfg.shared_inter,
             "score": cfg.score, "parallelism": f"replicas x{N}", "expert_kernel": expert_kernel,
             "expert_weights": "fp8 e4m3, 128x128 power-of-two block scales" if cfg.fp8 else cfg.dtype,
+            **({"fp8_gemm": "tokens on M" if fp8_tokens_on_m(cfg) else "tokens on N"} if cfg.fp8 else {}),
             "l2": l2}
 
 
@@ -496,6 +497,18 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     return ms, {k: v / max(n_rec, 1) for k, v in stage_ms.items()}, rec, ck
 
 
+FP8_FORM = {"value": "auto"}   # --fp8-kernel of this run
+
+
+def fp8_tokens_on_m(cfg):
+    """Whether moe_forward_fp8 runs this batch's expert GEMMs with the tokens
+    on the MMA's M side (more than 64 rows per expert on average, or forced)."""
+    form = FP8_FORM["value"]
+    if form != "auto":
+        return form == "tokens_on_m"
+    return cfg.T * cfg.topk > 64 * cfg.n_routed
+
+
 def rooflines(cfg, n_active, ms_step, per_kernel_ms, long_run):
     """The dominant kernel's roofline object and the layer roofline object."""
     pk, pk_kind = peaks()
@@ -512,7 +525,8 @@ def rooflines(cfg, n_active, ms_step, per_kernel_ms, long_run):
         roof = {"bound": "hbm", "achieved": up_b / t_up / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
         nominal = NOMINAL_PEAKS["hbm_gbs"]
     roof["frac"] = roof["achieved"] / roof["peak"]
-    kname = "grouped_fp8_kernel_up" if cfg.fp8 else "grouped_tc_kernel_up"
+    kname = ("grouped_fp8m_kernel_up" if fp8_tokens_on_m(cfg) else "grouped_fp8_kernel_up") if cfg.fp8 \
+        else "grouped_tc_kernel_up"
     roof.update({"traffic": traffic_for(kname, cfg.name),
                  "kernel": f"experts_up ({kname.replace('_up', '<UP>')})",
                  "algorithmic_flops": up_f, "algorithmic_bytes": up_b,
@@ -572,6 +586,7 @@ def ours_arm(a, D):
                                 "pair": M.MOE_EXPERT_KERNEL_TCGEN05_PAIR}[a.expert_kernel])
     M.moe_select_fp8_kernel({"auto": M.MOE_FP8_KERNEL_AUTO, "tokens_on_n": M.MOE_FP8_KERNEL_TOKENS_ON_N,
                              "tokens_on_m": M.MOE_FP8_KERNEL_TOKENS_ON_M}[a.fp8_kernel])
+    FP8_FORM["value"] = a.fp8_kernel
     S = Setup(cfg, dev)
     T = cfg.T
     launches = M.moe_forward_launch_count(cfg, T)
@@ -662,7 +677,7 @@ def ours_arm(a, D):
     others = None
     if N == 1 and not a.no_workloads and not a.tokens and not a.experts:
         others = {}
-        for name in ("v3_prefill", "v3_zipf", "softmax_nogroup", "v3_decode_fp8"):
+        for name in ("v3_prefill", "v3_zipf", "softmax_nogroup", "v3_decode_fp8", "v3_prefill_fp8"):
             if name == cfg.name:
                 continue
             o = inputs.CONFIGS[name]

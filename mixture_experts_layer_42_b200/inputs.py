@@ -98,6 +98,11 @@ CONFIGS = {
                                topk_groups=4, topk=8, moe_inter=2048, n_shared=1,
                                score="sigmoid", bias="normal", route_scale=2.5, dtype="bf16",
                                fp8=True),
+    # The prefill batch with its expert weights in the FP8 block-scaled layout.
+    "v3_prefill_fp8": MoEConfig("v3_prefill_fp8", T=8192, dim=7168, n_routed=256, n_groups=8,
+                                topk_groups=4, topk=8, moe_inter=2048, n_shared=1,
+                                score="sigmoid", bias="normal", route_scale=2.5, dtype="bf16",
+                                fp8=True),
 }
 
 # Zipf exponent of the skewed workload and the scale beta of its bias. Beta was
