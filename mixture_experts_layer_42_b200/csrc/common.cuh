@@ -336,11 +336,13 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
 // The same GEMMs with 128 token rows on the MMA's M side (gemm_fp8m.cu), for
 // batches with many rows per expert: UP reads the routed rows' codes in
 // expert order from xq_perm (scales xs_perm) and the shared MLP's from xq.
+// row_maps: the per-expert maps launch_row_maps(fp8 = true) wrote over xq_perm
+// and hq (an expert's last tile then reads zeros past its rows), or null.
 cudaError_t launch_grouped_fp8m(const moe_config& c, int64_t T, const Fp8Weights& w,
                                 const uint8_t* xq, const float* xs, const uint8_t* xq_perm,
                                 const float* xs_perm, const int32_t* offsets, uint8_t* hq,
                                 float* hsc, uint8_t* hsq, float* hss, void* y_perm, void* s,
-                                uint32_t* err, int num_sms, cudaStream_t st);
+                                const void* row_maps, uint32_t* err, int num_sms, cudaStream_t st);
 cudaError_t launch_grouped_simt(const moe_config& c, int64_t T, bool up, const GroupedArgs& g,
                                 cudaStream_t st);
 // Grouped tensor-core expert GEMM kernels (launch_grouped_tc `kind`).
@@ -364,9 +366,10 @@ cudaError_t launch_grouped_tc(bool up, int kind, int64_t Tk, int64_t T_sh, int E
 // A map over h [Tk, I] (at maps + E) and, when a_up is given, of the
 // up-projection's over a_up [Tk, D] (at maps), each with its row extent cut
 // at the expert's end; zeroes the up-projection's tile counter. Reads only
-// the offsets (a_up's rows need not be written yet).
+// the offsets (a_up's rows need not be written yet). fp8: maps over e4m3
+// rows for the FP8 token-on-M kernel (128-row boxes for every expert).
 cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, int D,
                             const int32_t* offsets, int E, void* maps, int* up_tile_ctr,
-                            cudaStream_t st);
+                            cudaStream_t st, bool fp8 = false);
 
 }  // namespace moe

@@ -93,6 +93,11 @@ struct Fp8mArgs {
   const float* ws1[2];   // weight scales [E, N/128, K/128] of tmW1
   const float* ws3[2];   // of tmW3
   const float* asc[2];   // the A rows' scales [rows, scale_stride(K)], in the A rows' order
+  // [E] copies of tmA[0] whose row extent ends at each expert's last row
+  // (written before the launch): an expert's last, partial tile reads zeros
+  // past its rows, which cost less power than the next expert's codes; null:
+  // tmA[0]
+  const CUtensorMap* row_maps;
   void* out[2];          // UP: quantized h [rows, N] e4m3; DOWN: bf16 [rows, N]
   float* out_scale[2];   // UP: h's scales [rows, scale_stride(N)]
   int n_out[2];
@@ -305,6 +310,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8m_kernel(const __grid_
       // its k-blocks and for a missing second block)
       const uint32_t w1a = ue8m0(nw[0]), w1b = ue8m0(nw[1]), w3a = ue8m0(nw[2]), w3b = ue8m0(nw[3]);
       const uint32_t tx = (uint32_t)(A_TILE + (two ? 2 : 1) * W_TILE);
+      const CUtensorMap* ta = &g.tmA[t.kind];
+      if (t.kind == 0 && t.rows < BM && g.row_maps != nullptr) {
+        ta = g.row_maps + t.e;
+        if (lane == 0) tmap_acquire(ta);
+      }
       for (int kb = 0; kb < kb_n; ++kb) {
         int w = 1;
         if (lane == 0) w = mbar_wait(&empty[s], ph ^ 1, abort_flag, g.err) ? 1 : 0;
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8m_kernel(const __grid_
           uint8_t* sa = tiles + s * STAGE_BYTES;
           uint8_t* sb = sa + A_TILE;
           mbar_expect_tx(&full[s], tx);
-          tma_load_2d(sa, &g.tmA[t.kind], &full[s], kb * QB, t.row0);
+          tma_load_2d(sa, ta, &full[s], kb * QB, t.row0);
           tma_load_3d(sb, &g.tmW1[t.kind], &full[s], kb * QB, t.n0, t.e);
           if (UP) tma_load_3d(sb + W_TILE, &g.tmW3[t.kind], &full[s], kb * QB, t.n0, t.e);
           else if (two) tma_load_3d(sb + W_TILE, &g.tmW1[t.kind], &full[s], kb * QB, t.n0 + QB, t.e);
@@ -557,7 +567,7 @@ cudaError_t launch_grouped_fp8m(const moe_config& c, int64_t T, const Fp8Weights
                                 const uint8_t* xq, const float* xs, const uint8_t* xq_perm,
                                 const float* xs_perm, const int32_t* offsets, uint8_t* hq,
                                 float* hsc, uint8_t* hsq, float* hss, void* y_perm, void* s,
-                                uint32_t* err, int num_sms, cudaStream_t st) {
+                                const void* row_maps, uint32_t* err, int num_sms, cudaStream_t st) {
   const int E = c.n_routed, D = c.dim, I = c.moe_inter, Is = c.shared_inter;
   const int64_t Tk = T * c.topk;
   const bool sh = Is > 0;
@@ -617,6 +627,8 @@ cudaError_t launch_grouped_fp8m(const moe_config& c, int64_t T, const Fp8Weights
     g.E = E;
     g.t_shared = sh ? (int)T : 0;
     g.err = err;
+    // UP's maps over xq_perm first, then DOWN's over hq
+    g.row_maps = row_maps ? static_cast<const CUtensorMap*>(row_maps) + (up ? 0 : E) : nullptr;
     const int bn = up ? QB : BN;   // output features per tile
     const int64_t bound = (int64_t)((n0 + bn - 1) / bn) * ((Tk + BM - 1) / BM + E) +
                           (sh ? (int64_t)((n1 + bn - 1) / bn) * ((T + BM - 1) / BM) : 0);

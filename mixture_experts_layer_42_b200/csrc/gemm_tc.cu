@@ -44,7 +44,7 @@
 // down-projection assigns them round-robin by CTA. Every pipeline wait is bounded
 // (1 s); on expiry the kernel raises the timeout bit of the error word, drains
 // what it has in flight, frees TMEM and returns.
-#include "tc_common.cuh"
+#include "fp8_common.cuh"
 
 namespace moe {
 
@@ -545,7 +545,7 @@ struct RowMapArgs {
 
 __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_constant__ RowMapArgs a,
                                                              const int32_t* __restrict__ offsets,
-                                                             int E, int* tile_ctr) {
+                                                             int E, int* tile_ctr, int swap_boxes) {
   // the up-projection, a programmatic dependent of this kernel when the
   // dispatch ran before it, may start now (it waits for this grid before its
   // routed tiles); this kernel is itself a programmatic dependent of the
@@ -563,8 +563,9 @@ __global__ void __launch_bounds__(256) build_row_maps_kernel(const __grid_consta
   if (lane == 0) {
     const int end = offsets[e + 1];
     // an expert with at most SWAP_ROWS rows: its only tile runs swapped, with
-    // a token box of tail_n(rows) rows; other experts keep BM-row boxes
-    const int tail = end - offsets[e] <= SWAP_ROWS ? end - offsets[e] : 0;
+    // a token box of tail_n(rows) rows; other experts keep BM-row boxes (all
+    // of them do for the FP8 kernel, which swaps no tile)
+    const int tail = swap_boxes && end - offsets[e] <= SWAP_ROWS ? end - offsets[e] : 0;
     asm volatile("tensormap.replace.tile.global_dim.shared::cta.b1024.b32 [%0], 1, %1;" ::"r"(
                      smem_u32(&sm[w])),
                  "r"(end > 0 ? end : 1)
@@ -593,17 +594,24 @@ int pipeline_stall() { return g_stall; }
 
 cudaError_t launch_row_maps(const void* h, int64_t Tk, int I, const void* a_up, int D,
                             const int32_t* offsets, int E, void* maps, int* up_tile_ctr,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool fp8) {
   RowMapArgs a;
   memset(&a, 0, sizeof(a));
-  if (!tc::map_2d(&a.base[0], h, (uint64_t)Tk, (uint64_t)I, BM)) return cudaErrorInvalidValue;
+  // bf16 rows (box 64 x 128) for the one-CTA kernel, e4m3 rows (box
+  // 128 x 128) for the FP8 token-on-M kernel
+  auto map = [&](CUtensorMap* m, const void* p, int K) {
+    return fp8 ? fp8::map_u8_tile(m, p, (uint64_t)Tk, (uint64_t)K, BM)
+               : tc::map_2d(m, p, (uint64_t)Tk, (uint64_t)K, BM);
+  };
+  if (!map(&a.base[0], h, I)) return cudaErrorInvalidValue;
   a.maps[0] = static_cast<CUtensorMap*>(maps) + E;
   if (a_up != nullptr) {
-    if (!tc::map_2d(&a.base[1], a_up, (uint64_t)Tk, (uint64_t)D, BM)) return cudaErrorInvalidValue;
+    if (!map(&a.base[1], a_up, D)) return cudaErrorInvalidValue;
     a.maps[1] = static_cast<CUtensorMap*>(maps);
   }
   dim3 grid((unsigned)((E + 7) / 8), a_up != nullptr ? 2u : 1u);
-  return launch_pdl(pdl_ok(), build_row_maps_kernel, grid, dim3(256), 0, st, a, offsets, E, up_tile_ctr);
+  return launch_pdl(pdl_ok(), build_row_maps_kernel, grid, dim3(256), 0, st, a, offsets, E, up_tile_ctr,
+                    fp8 ? 0 : 1);
 }
 
 // A: routed rows [Tk, K0] (or, for UP, the token rows gx [gT, K0] gathered

@@ -584,6 +584,15 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
   uint8_t* xq = at<uint8_t>(ws, F.xq);
   float* xs = at<float>(ws, F.xs);
   uint8_t* xq_perm = on_m ? at<uint8_t>(ws, F.xq_perm) : nullptr;
+  void* row_maps = at<void>(ws, L.row_maps);
+  if (on_m) {
+    // per-expert maps over the routed rows of x and h (the tile counter the
+    // kernel also zeroes is not used on this path)
+    int* ctr = reinterpret_cast<int*>(static_cast<uint8_t*>(row_maps) + (size_t)2 * c.n_routed * 128);
+    if (launch_row_maps(at<uint8_t>(ws, F.hq), T * c.topk, c.moe_inter, xq_perm, c.dim, offsets,
+                        c.n_routed, row_maps, ctr, s, true) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   if (launch_quant_rows(c, x, T, c.dim, xq, xs, fp8_stride_host(c.dim), s, pos,
                         at<float>(ws, F.xs_perm), xq_perm) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -596,7 +605,7 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
   const cudaError_t ge =
       on_m ? launch_grouped_fp8m(c, T, fw, xq, xs, xq_perm, at<float>(ws, F.xs_perm), offsets,
                                  at<uint8_t>(ws, F.hq), at<float>(ws, F.hs), at<uint8_t>(ws, F.hsq),
-                                 at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf, err,
+                                 at<float>(ws, F.hss), at<void>(ws, L.y_perm), sbuf, row_maps, err,
                                  num_sms_current(), s)
            : launch_grouped_fp8(c, T, fw, xq, xs, at<float>(ws, F.xs_perm), src, offsets,
                                 at<uint8_t>(ws, F.hq), at<float>(ws, F.hs), at<uint8_t>(ws, F.hsq),
