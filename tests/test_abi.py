@@ -89,6 +89,10 @@ def test_bad_sizes_and_pointers(M):
     assert M.raw_status("moe_workspace_init", None, 0, None) == -1
     assert M.raw_status("moe_check_error", ctypes.c_void_p(0x1001), None) == -1
     assert M.raw_status("moe_select_expert_kernel", 5) == -1
+    assert M.raw_status("moe_select_fp8_kernel", 3) == -1
+    assert M.raw_status("moe_select_fp8_kernel", -1) == -1
+    for which in (M.MOE_FP8_KERNEL_TOKENS_ON_M, M.MOE_FP8_KERNEL_TOKENS_ON_N, M.MOE_FP8_KERNEL_AUTO):
+        assert M.raw_status("moe_select_fp8_kernel", which) == 0
 
 
 def test_workspace_too_small_is_rejected_before_launch(M):
