@@ -393,7 +393,8 @@ MOE_API moe_status moe_select_fp8_kernel(int32_t which);
  * has its first CTA wait, before it issues anything, on a barrier phase that
  * nothing completes:
  *   1  the up-projection of every bf16 layer on the one-CTA tensor-core
- *      kernel (the rows of that CTA's tiles are not written);
+ *      kernel, and of every FP8 layer in either form (the rows of that
+ *      CTA's tiles are not written);
  *   2  the tensor-core router logits of every bf16 layer (that CTA's partial
  *      sums are not written).
  * The wait runs out after its 1 s limit; the launch then takes the abort

@@ -121,6 +121,10 @@ struct Fp8Args {
   const int32_t* offsets;
   int E;
   int t_shared;
+  // Test hook (moe_debug_stall_pipeline): CTA 0's MMA thread first waits on
+  // a barrier phase that nothing completes, so that wait runs out (1 s)
+  // before anything is issued, and the launch takes its abort path.
+  int stall;
   uint32_t* err;
 };
 
@@ -402,6 +406,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       int s = 0, groups = 0, hint = 0;
       uint32_t ph = 0, tsa = 0;
       bool ok = true;
+      // test hook: a wait that runs out (the drain barrier is committed only
+      // after the tile loop), before any MMA is issued
+      if (g.stall && blockIdx.x == 0 && !mbar_wait(drain, 0, abort_flag, g.err)) ok = false;
       for (int i = blockIdx.x, lt = 0; ok && i < S.total; i += gridDim.x, ++lt) {
         const Tile t = decode(S, i, hint);
         const int kb_n = g.kdim[t.kind] / QB;
@@ -776,6 +783,7 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
     g.E = E;
     g.t_shared = sh ? (int)T : 0;
     g.err = err;
+    g.stall = up && pipeline_stall() == STALL_EXPERTS_UP ? 1 : 0;
     const int bn = up ? TileN<true>::BN : TileN<false>::BN;   // output features per tile
     const int64_t bound = (int64_t)((n0 + bn - 1) / bn) * ((Tk + NT - 1) / NT + E) +
                           (sh ? (int64_t)((n1 + bn - 1) / bn) * ((T + NT - 1) / NT) : 0);

@@ -43,3 +43,32 @@ def test_pipeline_wait_runs_out_and_is_reported():
     # the same context: the next forward is exact
     err, r, nt = forward_parity(L)
     assert err < 2e-2
+
+
+@pytest.mark.parametrize("form", ["tokens_on_n", "tokens_on_m"])
+def test_fp8_pipeline_wait_runs_out_and_is_reported(form):
+    # the same hook on the FP8 up-projection, in each of its two forms
+    from tests.test_gpu_fp8 import FORMS, Fp8Layer, _parity, small
+    cfg = small(T=300, seed=5)
+    F = Fp8Layer(Layer(cfg))
+    M.moe_select_fp8_kernel(FORMS[form])
+    try:
+        L = F.L
+        ws = M.alloc_workspace_fp8(cfg, L.T)
+        y = torch.empty(L.T, cfg.dim, dtype=torch.bfloat16, device="cuda")
+        M.moe_debug_stall_pipeline(1)
+        try:
+            t0 = time.time()
+            M.moe_forward_fp8(cfg, L.x, L.w_r, L.bias, F.fw, y, ws)
+            status = M.moe_check_error(ws)      # synchronises
+            elapsed = time.time() - t0
+        finally:
+            M.moe_debug_stall_pipeline(0)
+        assert status == M.MOE_ERR_TIMEOUT
+        assert 0.9 < elapsed < 30
+        assert M.moe_check_error(ws) == M.MOE_OK
+        # the same context: the next FP8 forward matches the oracle
+        err, *_ = _parity(cfg)
+        assert err < 2e-2
+    finally:
+        M.moe_select_fp8_kernel(M.MOE_FP8_KERNEL_AUTO)
