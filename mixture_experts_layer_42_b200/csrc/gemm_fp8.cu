@@ -549,7 +549,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
 }
 
 // Rows [R, K] (act) to e4m3 with one power-of-two scale per 1 x 128 block:
-// one warp per block, 4 elements per lane.
+// one warp per two blocks of a row, a half-warp per block, 8 elements (one or
+// two 16-byte loads, one 8-byte store of codes) per lane.
 // With pos, each block's scale is also written to the k permuted rows of its
 // row's (token, slot) pairs (scale_perm, for the up-projection's routed rows;
 // pairs with pos < 0 are skipped), and with q_perm its codes too (the
@@ -566,32 +567,54 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T* __restrict__ a
   asm volatile("griddepcontrol.launch_dependents;");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int kbn = K / QB;
-  const int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int pairs = (kbn + 1) / 2;     // block pairs per row
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
-  if (blk >= R * kbn) return;
-  const int64_t r = blk / kbn;
-  const int kb = (int)(blk % kbn);
-  const T* p = a + r * K + kb * QB + lane * 4;
-  float v[4];
+  if (w >= R * pairs) return;          // whole warps
+  const int64_t r = w / pairs;
+  const int kb = (int)(w % pairs) * 2 + (lane >> 4);   // this half-warp's block
+  const int sl = lane & 15;                            // elements 8 sl .. 8 sl + 7 of it
+  const bool active = kb < kbn;                        // the second block of an odd row end: none
+  float v[8];
+  if (active) {
+    const T* p = a + r * K + kb * QB + sl * 8;
+    Vec16<T> x0;
+    x0.raw = reinterpret_cast<const uint4*>(p)[0];
+    x0.to_float(v);
+    if (Vec16<T>::N == 4) {
+      Vec16<T> x1;
+      x1.raw = reinterpret_cast<const uint4*>(p)[1];
+      x1.to_float(v + 4);
+    }
+  } else {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = to_f32(p[i]);
-  float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  }
+  float m = 0.f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));  // within the half
   const int se = block_exp(m);
-  uint32_t packed = 0;
+  uint32_t c0 = 0, c1 = 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) packed |= (uint32_t)to_e4m3(ldexpf(v[i], -se)) << (8 * i);
-  reinterpret_cast<uint32_t*>(q + r * K + kb * QB)[lane] = packed;
+  for (int i = 0; i < 4; ++i) {
+    c0 |= (uint32_t)to_e4m3(ldexpf(v[i], -se)) << (8 * i);
+    c1 |= (uint32_t)to_e4m3(ldexpf(v[4 + i], -se)) << (8 * i);
+  }
+  const uint2 codes = make_uint2(c0, c1);
   const float sc = ldexpf(1.f, se);
-  if (lane == 0) scale[r * sstride + kb] = sc;
+  if (active) {
+    reinterpret_cast<uint2*>(q + r * K + kb * QB)[sl] = codes;
+    if (sl == 0) scale[r * sstride + kb] = sc;
+  }
   if (pos != nullptr) {
-    const int p = lane < k ? pos[r * k + lane] : -1;
-    if (p >= 0) scale_perm[(int64_t)p * sstride + kb] = sc;
-    if (q_perm != nullptr) {
-      for (int j = 0; j < k; ++j) {   // k <= 32
-        const int pj = __shfl_sync(0xffffffffu, p, j);
-        if (pj >= 0) reinterpret_cast<uint32_t*>(q_perm + (int64_t)pj * K + kb * QB)[lane] = packed;
+    const int p = lane < k ? pos[r * k + lane] : -1;   // k <= 32
+    for (int j = 0; j < k; ++j) {
+      const int pj = __shfl_sync(0xffffffffu, p, j);
+      if (pj >= 0 && active) {
+        if (sl == 0 && scale_perm != nullptr) scale_perm[(int64_t)pj * sstride + kb] = sc;
+        if (q_perm != nullptr) reinterpret_cast<uint2*>(q_perm + (int64_t)pj * K + kb * QB)[sl] = codes;
       }
     }
   }
@@ -675,7 +698,7 @@ bool map_u8_weights(CUtensorMap* m, const void* ptr, uint64_t E, uint64_t N, uin
 cudaError_t launch_quant_rows(const moe_config& c, const void* a, int64_t R, int K, uint8_t* q,
                               float* scale, int sstride, cudaStream_t st, const int32_t* pos,
                               float* scale_perm, uint8_t* q_perm) {
-  const int64_t warps = R * (K / QB);
+  const int64_t warps = R * ((K / QB + 1) / 2);
   if (warps == 0) return cudaSuccess;
   if (sstride <= 0) sstride = K / QB;
   const unsigned blocks = (unsigned)ceil_div<int64_t>(warps * 32, 256);
