@@ -15,7 +15,8 @@
 // block; two per stage, UP's w1 and w3 rows or 256 of DOWN's w2 rows) and up
 // to NT = 32 tokens of one expert on its N side, so a decode batch (a few
 // tokens per expert) does little MMA work while it streams the active
-// experts' weights at half the bytes of bf16. Every MMA is block-scaled: per
+// experts' weights at half the bytes of bf16. (Batches with more rows per
+// expert run the token-on-M form of gemm_fp8m.cu.) Every MMA is block-scaled: per
 // 32-deep slice of K it multiplies each weight row by its UE8M0 scale and each
 // token by its own, so one fp32 TMEM accumulator sums the whole K,
 //   sum[f, t] = sum_kb s_w(e, f/128, kb) s_x(t, kb) sum_{k in kb} q_w[f, k] q_x[t, k]
@@ -816,7 +817,7 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
         e = cudaFuncSetAttribute(grouped_fp8_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)FSMEM);
         if (e != cudaSuccess) return e;
-        // a programmatic dependent of the row quantization (or the scale gather)
+        // a programmatic dependent of the row quantization
         e = launch_pdl(pdl_ok(), grouped_fp8_kernel<true>, dim3(grid), dim3(NTHREADS), FSMEM, st, g);
         if (e != cudaSuccess) return e;
       } else {
