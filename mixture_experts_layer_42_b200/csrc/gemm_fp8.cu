@@ -172,9 +172,10 @@ __device__ __forceinline__ Tile decode(const Sched& S, int i, int& hint) {
 
 template <bool UP>
 __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_constant__ Fp8Args g) {
-  // the kernel after this one (the combine, after the down-projection) may
-  // launch now; it waits for this grid before it reads the outputs
-  asm volatile("griddepcontrol.launch_dependents;");
+  // DOWN: the combine after it may launch now (it waits for this grid
+  // before it reads the outputs). UP lets the down-projection launch only
+  // after its own prologue (below), once it has waited for its predecessors.
+  if (!UP) asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int FSTAGES = Ring<UP>::STAGES;
@@ -212,7 +213,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // a programmatic dependent (up-projection): wait for the kernel before it
     // before anything it or its predecessors wrote is read (the offsets here;
     // src, the scales and x's codes after the __syncthreads below)
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // (DOWN, a programmatic dependent of the up-projection, reads here only
+    // what was complete before that grid let it launch, the offsets: it
+    // waits for h in its producer, after prefetching its first weight tiles)
+    if (UP) asm volatile("griddepcontrol.wait;" ::: "memory");
     // token chunks per expert and their exclusive prefix
     const int per = (E + 31) / 32;
     int lsum = 0;
@@ -251,6 +255,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // UP: every thread of the CTA is past the wait for the kernels before it,
+  // so a dependent down-projection may read what they wrote (the offsets)
+  // before it waits for this grid
+  if (UP) asm volatile("griddepcontrol.launch_dependents;");
 
   Sched S;
   S.P = P;
@@ -274,6 +282,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     int hint = 0, hint_next = 0;            // experts of the last tile decoded, this and next
     uint32_t ph = 0;
     bool ok = true;
+    if (!UP) {
+      // the first tile's leading weight k-blocks into L2 while the
+      // up-projection finishes, then wait for it (h and its scales)
+      if (lane == 0 && (int)blockIdx.x < S.total) {
+        int h0 = 0;
+        const Tile t0 = decode(S, blockIdx.x, h0);
+        const int kb_n = g.kdim[t0.kind] / QB;
+        const bool two0 = t0.n0 + QB < g.n_out[t0.kind];
+        const int n_pf = min(kb_n, DOWN_PREFETCH_KB_BYTES / (2 * W_BYTES));
+        for (int kb = 0; kb < n_pf; ++kb) {
+          tma_prefetch_3d(&g.tmW1[t0.kind], kb * QB, t0.n0, t0.e);
+          if (two0) tma_prefetch_3d(&g.tmW1[t0.kind], kb * QB, t0.n0 + QB, t0.e);
+        }
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
     if (lane == 0 && (int)blockIdx.x < S.total) {   // the first tile's token scales
       int h0 = 0;
       const Tile t0 = decode(S, blockIdx.x, h0);
@@ -824,7 +848,9 @@ cudaError_t launch_grouped_fp8(const moe_config& c, int64_t T, const Fp8Weights&
         e = cudaFuncSetAttribute(grouped_fp8_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)FSMEM);
         if (e != cudaSuccess) return e;
-        grouped_fp8_kernel<false><<<grid, NTHREADS, FSMEM, st>>>(g);
+        // a programmatic dependent of the up-projection
+        e = launch_pdl(pdl_ok(), grouped_fp8_kernel<false>, dim3(grid), dim3(NTHREADS), FSMEM, st, g);
+        if (e != cudaSuccess) return e;
       }
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -151,9 +151,10 @@ __device__ __forceinline__ float silu_fast(float u) { return u / (1.0f + __expf(
 
 template <bool UP>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid_constant__ TcArgs g) {
-  // the kernel after this one (the combine, after the down-projection) may
-  // launch now; it waits for this grid before it reads the outputs
-  asm volatile("griddepcontrol.launch_dependents;");
+  // DOWN: the combine after it may launch now (it waits for this grid
+  // before it reads the outputs). UP lets the down-projection launch only
+  // after its own prologue (below), once it has waited for its predecessors.
+  if (!UP) asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* tiles = base;
@@ -188,7 +189,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     // one completes: wait for it before anything it wrote is read (the
     // offsets here; src, the row maps and the tile counter after the
     // __syncthreads below). Returns at once for an ordinary launch.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // DOWN, a programmatic dependent of the up-projection, reads here only
+    // what was complete before that grid let it launch (the offsets; the row
+    // maps below): it waits for h in its producer, after prefetching the
+    // first weight tiles.
+    if (UP) asm volatile("griddepcontrol.wait;" ::: "memory");
     // m-tiles per expert and their exclusive prefix
     const int per = (E + 31) / 32;
     int lsum = 0;
@@ -227,6 +232,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // UP: every thread of the CTA is past the wait for the kernels before it,
+  // so a dependent down-projection may read what they wrote (the offsets,
+  // the row maps) before it waits for this grid
+  if (UP) asm volatile("griddepcontrol.launch_dependents;");
 
   Sched S;
   S.P = P;
@@ -251,6 +260,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
     bool ok = true;
     TileQueue Q;
     const bool dyn = g.tile_ctr != nullptr;
+    if (!UP) {
+      // the first tile's leading weight k-blocks into L2 while the
+      // up-projection finishes, then wait for it (h)
+      if (lane == 0 && (int)blockIdx.x < S.total) {
+        const Tile t0 = decode(S, blockIdx.x);
+        const int kb_n = (g.kdim[t0.kind] + BK - 1) / BK;
+        const int n_pf = min(kb_n, DOWN_PREFETCH_KB_BYTES / B_TILE);
+        for (int kb = 0; kb < n_pf; ++kb) tma_prefetch_3d(&g.tmB1[t0.kind], kb * BK, t0.n0, t0.e);
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
     // the next tile is claimed a few k-blocks before the current one ends,
     // so the atomic's round trip overlaps the current tile's loads
     int next = 0;

@@ -142,10 +142,12 @@ moe_status run_experts(const moe_config& c, int64_t T, const void* x_perm, const
                           x_perm ? nullptr : src, T, kind == TC_ROWS ? row_maps : nullptr, ctr, err,
                           num_sms_current(), st, pdl);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
+    // the down-projection as a programmatic dependent of the up-projection:
+    // it prefetches its first weight tiles while the up-projection finishes
     e = launch_grouped_tc(false, kind, Tk, sh ? T : 0, c.n_routed, h, hs, w2, nullptr, ws2, nullptr,
                           c.dim, c.moe_inter, c.dim, c.shared_inter, y_perm, s, offsets, nullptr,
                           nullptr, 0, kind == TC_ROWS ? maps_down : nullptr, nullptr, err,
-                          num_sms_current(), st, false);
+                          num_sms_current(), st, kind == TC_ROWS && !stage_timing_active());
     return cuda_status(e);
   }
   if (place != nullptr && launch_dispatch_place(*place, st) != cudaSuccess)

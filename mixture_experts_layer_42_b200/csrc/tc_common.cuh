@@ -124,6 +124,19 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* tm, ui
       : "memory");
 }
 
+// One box of a 3D tensor into L2 only (no shared-memory destination, no
+// barrier): the down-projection's first weight tiles, fetched while the
+// up-projection before it finishes.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* tm, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tm), "r"(c0),
+               "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// k-blocks of a down-projection CTA's first tile prefetched into L2 before
+// it waits for the up-projection (256 KB per CTA, ~38 MB over the GPU).
+constexpr int DOWN_PREFETCH_KB_BYTES = 256 * 1024;
+
 // Four rows of a 2D tensor (a map whose box is 64 elements x 1 row) into
 // shared memory as one 4-row, 512-byte piece of a 128-byte-swizzled tile: row
 // coordinates r0..r3 may be anything (an out-of-range row reads zeros), the
