@@ -210,12 +210,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    // a programmatic dependent (up-projection): wait for the kernel before it
-    // before anything it or its predecessors wrote is read (the offsets here;
-    // src, the scales and x's codes after the __syncthreads below)
-    // (DOWN, a programmatic dependent of the up-projection, reads here only
-    // what was complete before that grid let it launch, the offsets: it
-    // waits for h in its producer, after prefetching its first weight tiles)
+    // UP, a programmatic dependent of the row quantization: wait for it
+    // before anything it or the kernels before it wrote is read (the offsets
+    // here; src, the scales and x's codes after the __syncthreads below).
+    // DOWN, a programmatic dependent of the up-projection, reads here only
+    // what was complete before that grid let it launch (the offsets); it
+    // waits for h in its producer, after prefetching its first weight tiles.
     if (UP) asm volatile("griddepcontrol.wait;" ::: "memory");
     // token chunks per expert and their exclusive prefix
     const int per = (E + 31) / 32;

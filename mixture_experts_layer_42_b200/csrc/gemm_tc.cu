@@ -184,14 +184,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_tc_kernel(const __grid
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    // Launched as a programmatic dependent of the kernel before it (the
-    // dispatch or the row-map kernel), this grid may be running before that
-    // one completes: wait for it before anything it wrote is read (the
+    // UP, launched as a programmatic dependent of the kernel before it (the
+    // dispatch or the row-map kernel), may be running before that one
+    // completes: it waits for it before anything it wrote is read (the
     // offsets here; src, the row maps and the tile counter after the
-    // __syncthreads below). Returns at once for an ordinary launch.
+    // __syncthreads below). The wait returns at once for an ordinary launch.
     // DOWN, a programmatic dependent of the up-projection, reads here only
-    // what was complete before that grid let it launch (the offsets; the row
-    // maps below): it waits for h in its producer, after prefetching the
+    // what was complete before that grid let it launch (the offsets; later
+    // the row maps); it waits for h in its producer, after prefetching its
     // first weight tiles.
     if (UP) asm volatile("griddepcontrol.wait;" ::: "memory");
     // m-tiles per expert and their exclusive prefix
