@@ -152,11 +152,17 @@ def test_fp8_forward_matches_oracle(kw, form):
                                      moe_inter=384),
                                 dict(T=700, n_routed=4, n_groups=1, topk_groups=1, topk=1, n_shared=0),
                                 dict(T=513, dim=256, moe_inter=128, n_routed=2, n_groups=1,
+                                     topk_groups=1, topk=2),
+                                dict(T=600, dim=128, moe_inter=128, n_routed=4, n_groups=1,
+                                     topk_groups=1, topk=2),
+                                dict(T=300, dim=8192, moe_inter=256, n_routed=4, n_groups=1,
                                      topk_groups=1, topk=2)])
 def test_fp8_forward_many_rows_per_expert(kw, form):
     # experts with several 128-row tiles and ragged last tiles; a layer with
     # dim an odd multiple of 128 (its last down-projection tile one weight
-    # block wide) and every expert taking every token
+    # block wide); every expert taking every token; the smallest and the
+    # largest reduction depth the FP8 layout allows (one 128-deep k-block,
+    # and 64 of them)
     err, *_ = _parity(small(**kw))
     assert err < 2e-2
 
