@@ -102,3 +102,28 @@ def test_l2_note_states_how_the_timed_loop_meets_l2():
     # the rest of the roofline inputs the GPU arm builds its line from
     flops, byts, t, bound = bench.layer_roofline(inputs.CONFIGS["v3_decode"], 158, bench.NOMINAL_PEAKS)
     assert bound == "hbm" and t > 0
+
+
+def test_fp8_rooflines_use_twice_the_bf16_peak_and_name_the_form():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixture_experts_layer_42_b200 import inputs
+    pk, _ = bench.peaks()
+    dec, pre = inputs.CONFIGS["v3_decode_fp8"], inputs.CONFIGS["v3_prefill_fp8"]
+    # the form the library picks: tokens on M above 64 rows per expert on average
+    assert not bench.fp8_tokens_on_m(dec) and bench.fp8_tokens_on_m(pre)
+    assert bench.config_dict(dec, 1, "auto", "")["fp8_gemm"] == "tokens on N"
+    assert bench.config_dict(pre, 1, "auto", "")["fp8_gemm"] == "tokens on M"
+    # e4m3 products at twice the bf16 peak, weights at one byte (and a scale per block)
+    f16, b16, t16, _ = bench.layer_roofline(inputs.CONFIGS["v3_prefill"], 229, pk)
+    f8, b8, t8, bound = bench.layer_roofline(pre, 229, pk)
+    assert f8 == f16 and bound == "tensor" and b8 < 0.55 * b16
+    t_router = 2 * pre.T * pre.dim * pre.n_routed / (pk["bf16_tflops"] * 1e12)   # stays bf16
+    assert abs(t8 - (t_router + (t16 - t_router) / 2)) < 1e-12
+    up_f, _ = bench.up_kernel_work(pre, 229)
+    roof, _ = bench.rooflines(pre, 229, 5.6, {"experts_up": 3.0}, False)
+    assert roof["bound"] == "tensor" and roof["peak"] == 2 * pk["bf16_tflops"]
+    assert abs(roof["achieved"] - up_f / 3e-3 / 1e12) < 1e-6
+    assert roof["kernel"] == "experts_up (grouped_fp8m_kernel<UP>)"
+    roof, _ = bench.rooflines(dec, 158, 1.13, {"experts_up": 0.72}, False)
+    assert roof["bound"] == "hbm" and roof["kernel"] == "experts_up (grouped_fp8_kernel<UP>)"
