@@ -178,7 +178,11 @@ MOE_API moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_p
  * dependent of the dispatch's last kernel (cudaLaunchKernelEx with
  * programmatic stream serialization): its CTAs start, and take any shared-
  * expert tiles, while that kernel finishes, and wait for it (griddepcontrol)
- * before their first routed tile. */
+ * before their first routed tile. The down-projection is in turn a
+ * programmatic dependent of the up-projection: its CTAs start as the
+ * up-projection's finish, prefetch their first weight tiles into L2 and wait
+ * for h. Every kernel of the chain waits for its predecessor before it reads
+ * what that grid wrote, so results do not depend on the overlap. */
 MOE_API moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const void* w_router,
                        const float* bias, const void* w1, const void* w3, const void* w2,
                        const void* ws1, const void* ws3, const void* ws2, void* y,
