@@ -502,11 +502,11 @@ FP8_FORM = {"value": "auto"}   # --fp8-kernel of this run
 
 def fp8_tokens_on_m(cfg):
     """Whether moe_forward_fp8 runs this batch's expert GEMMs with the tokens
-    on the MMA's M side (more than 64 rows per expert on average, or forced)."""
+    on the MMA's M side (more than 16 rows per expert on average, or forced)."""
     form = FP8_FORM["value"]
     if form != "auto":
         return form == "tokens_on_m"
-    return cfg.T * cfg.topk > 64 * cfg.n_routed
+    return cfg.T * cfg.topk > 16 * cfg.n_routed
 
 
 def rooflines(cfg, n_active, ms_step, per_kernel_ms, long_run):

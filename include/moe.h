@@ -275,7 +275,7 @@ MOE_API moe_status moe_workspace_size_fp8(const moe_config* cfg, int64_t T, size
  * moe_forward. Workspace of moe_workspace_size_fp8() bytes, initialised by
  * moe_workspace_init(). bf16 layers only.
  * Two forms of the expert GEMMs compute the same sums (see
- * moe_select_fp8_kernel): for batches of at most 64 rows per expert on
+ * moe_select_fp8_kernel): for batches of at most 16 rows per expert on
  * average, the weights on the MMA's M side and up to 32 tokens of an expert on
  * its N side (each weight tile streamed once per 32 tokens); above that, 128
  * token rows on M and 256 weight rows on N, the routed rows' codes written in
@@ -379,7 +379,7 @@ MOE_API moe_status moe_select_expert_kernel(int32_t which);
 
 /* Which form runs the expert GEMMs of moe_forward_fp8, process-wide (for
  * checks and measurement):
- *   AUTO (default)  by the batch: tokens on N for at most 64 (token, slot)
+ *   AUTO (default)  by the batch: tokens on N for at most 16 (token, slot)
  *                   rows per expert on average, tokens on M above;
  *   TOKENS_ON_N     weights on the MMA's M side, up to 32 tokens on N;
  *   TOKENS_ON_M     128 token rows on M, 256 weight rows on N.

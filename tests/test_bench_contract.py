@@ -110,7 +110,7 @@ def test_fp8_rooflines_use_twice_the_bf16_peak_and_name_the_form():
     from mixture_experts_layer_42_b200 import inputs
     pk, _ = bench.peaks()
     dec, pre = inputs.CONFIGS["v3_decode_fp8"], inputs.CONFIGS["v3_prefill_fp8"]
-    # the form the library picks: tokens on M above 64 rows per expert on average
+    # the form the library picks: tokens on M above 16 rows per expert on average
     assert not bench.fp8_tokens_on_m(dec) and bench.fp8_tokens_on_m(pre)
     assert bench.config_dict(dec, 1, "auto", "")["fp8_gemm"] == "tokens on N"
     assert bench.config_dict(pre, 1, "auto", "")["fp8_gemm"] == "tokens on M"
