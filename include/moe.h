@@ -167,8 +167,8 @@ MOE_API moe_status moe_combine(const moe_config* cfg, int64_t T, const void* y_p
 /* The whole layer (MoE.forward): gate, dispatch, experts and combine chained
  * on `stream` with no host synchronisation. y [T, D] (act). weights_out
  * [T, k] and idx_out [T, k] may be NULL; when given they receive the routing.
- * For batches of at most 64 routed rows per expert on average (T * k <=
- * 64 * n_routed: decode) and for fp32 layers, the experts read the routed
+ * For batches of at most 16 routed rows per expert on average (T * k <=
+ * 16 * n_routed: decode) and for fp32 layers, the experts read the routed
  * token rows straight from x (as moe_experts_grouped_gather does) and no
  * permuted copy of x is made. Larger bf16 batches, and the CTA-pair expert
  * kernel, read an expert-contiguous copy that dispatch writes into the

@@ -213,9 +213,12 @@ struct TimedCall {
 };
 
 // Average rows per expert up to which moe_forward gathers the up-projection's
-// rows from x instead of copying them (the swapped-tile limit of the one-CTA
-// tensor-core kernel).
-constexpr int64_t kGatherRows = 64;
+// rows from x instead of copying them. Measured at the DeepSeek-V3 shape: the
+// two take the same time at 16 rows per expert (T = 512), and the copy is
+// faster above (T = 1024: 2.99 vs 3.51 ms per step; T = 2048: 3.56 vs 4.91),
+// where experts run multi-row or 128-row tiles whose gathers bound the stage
+// rate.
+constexpr int64_t kGatherRows = 16;
 
 // Average rows per expert above which moe_forward_fp8 runs its expert GEMMs
 // with the tokens on the MMA's M side (the crossover measured at the
@@ -398,8 +401,8 @@ moe_status moe_forward(const moe_config* cfg, int64_t T, const void* x, const vo
   // Measured on B200 at the DeepSeek-V3 shape: with 128-row tiles the 32
   // gathers per stage bound the up-projection by the TMA's copy rate (10.9
   // against 4.8 ms at T = 8192), while batches of at most kGatherRows rows per
-  // expert (decode) run their few rows as swapped tiles and gather 4 to 16 rows
-  // per stage at no cost. So batches that average more rows per expert, and
+  // expert on average (decode) run their few rows as swapped tiles and gather
+  // 4 to 16 rows per stage at no cost. So batches that average more rows per expert, and
   // the CTA-pair option, take the copy; it lives in y_perm's space, which is
   // free until the down-projection writes it.
   const bool big = T * (int64_t)c.topk > (int64_t)kGatherRows * c.n_routed;
