@@ -279,9 +279,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
     // its row of each stage's scale-factor bytes: the weight block's scale
     // (the same for all 128 weight rows of the tile) and its token's.
     int s = 0, issued = 0, scopies = 0;
-    int hint = 0, hint_next = 0;            // experts of the last tile decoded, this and next
+    int hint = 0, hint_next = 0, hint_w = 0;  // experts of the last tile decoded: this, next, scales
     uint32_t ph = 0;
     bool ok = true;
+    // the weight-block scales of a tile, k-blocks lane and lane + 32 (1.0 past
+    // its k-blocks and for a missing second block), loaded a tile ahead
+    float nw[4];
+    auto load_wscales = [&](const Tile& tt) {
+      const int kbn = g.kdim[tt.kind] / QB;
+      const int nbw = g.n_out[tt.kind] / QB;
+      const bool two_t = UP || tt.n0 + QB < g.n_out[tt.kind];
+      const float* pw1 = g.ws1[tt.kind] + ((int64_t)tt.e * nbw + tt.n0 / QB) * kbn;
+      const float* pw3 = UP ? g.ws3[tt.kind] + ((int64_t)tt.e * nbw + tt.n0 / QB) * kbn : pw1 + kbn;
+      nw[0] = lane < kbn ? __ldg(pw1 + lane) : 1.f;
+      nw[1] = lane + 32 < kbn ? __ldg(pw1 + lane + 32) : 1.f;
+      nw[2] = two_t && lane < kbn ? __ldg(pw3 + lane) : 1.f;
+      nw[3] = two_t && lane + 32 < kbn ? __ldg(pw3 + lane + 32) : 1.f;
+    };
+    if ((int)blockIdx.x < S.total) load_wscales(decode(S, blockIdx.x, hint_w));
     if (!UP) {
       // the first tile's leading weight k-blocks into L2 while the
       // up-projection finishes, then wait for it (h and its scales)
@@ -315,17 +330,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) grouped_fp8_kernel(const __grid_c
       // the second weight tile: UP w3's rows, DOWN the next 128 rows of w2
       // (none in a DOWN tile at the end of an odd number of row blocks)
       const bool two = UP || t.n0 + QB < g.n_out[t.kind];
-      // the tile's weight scales as UE8M0 bytes, k-blocks lane and lane + 32
-      const int nbw = g.n_out[t.kind] / QB;
-      const float* pw1 = g.ws1[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n;
-      const uint32_t w1a = lane < kb_n ? ue8m0(__ldg(pw1 + lane)) : 127u;
-      const uint32_t w1b = lane + 32 < kb_n ? ue8m0(__ldg(pw1 + lane + 32)) : 127u;
-      uint32_t w3a = 127u, w3b = 127u;
-      if (two) {
-        const float* pw3 = UP ? g.ws3[t.kind] + ((int64_t)t.e * nbw + t.n0 / QB) * kb_n : pw1 + kb_n;
-        w3a = lane < kb_n ? ue8m0(__ldg(pw3 + lane)) : 127u;
-        w3b = lane + 32 < kb_n ? ue8m0(__ldg(pw3 + lane + 32)) : 127u;
-      }
+      // the tile's weight scales as UE8M0 bytes (loaded a tile ahead), then
+      // the next tile's loads
+      const uint32_t w1a = ue8m0(nw[0]), w1b = ue8m0(nw[1]), w3a = ue8m0(nw[2]), w3b = ue8m0(nw[3]);
+      if (i + (int)gridDim.x < S.total) load_wscales(decode(S, i + gridDim.x, hint_w));
       // this tile's token scales (copied a tile ahead), then the next tile's
       // copy into the other slot (its last reader, the previous tile's loop
       // below, is done: the warp has synchronised since)
