@@ -497,16 +497,12 @@ def device_timed(S, D, steps, warmup, uuid, clocks_on):
     return ms, {k: v / max(n_rec, 1) for k, v in stage_ms.items()}, rec, ck
 
 
-FP8_FORM = {"value": "auto"}   # --fp8-kernel of this run
-
-
 def fp8_tokens_on_m(cfg):
     """Whether moe_forward_fp8 runs this batch's expert GEMMs with the tokens
-    on the MMA's M side (more than 16 rows per expert on average, or forced)."""
-    form = FP8_FORM["value"]
-    if form != "auto":
-        return form == "tokens_on_m"
-    return cfg.T * cfg.topk > 16 * cfg.n_routed
+    on the MMA's M side, as the library resolves it (its selection, or by the
+    average rows per expert)."""
+    from mixture_experts_layer_42_b200 import binding as M
+    return M.moe_fp8_kernel_for(cfg, cfg.T) == M.MOE_FP8_KERNEL_TOKENS_ON_M
 
 
 def rooflines(cfg, n_active, ms_step, per_kernel_ms, long_run):
@@ -586,7 +582,6 @@ def ours_arm(a, D):
                                 "pair": M.MOE_EXPERT_KERNEL_TCGEN05_PAIR}[a.expert_kernel])
     M.moe_select_fp8_kernel({"auto": M.MOE_FP8_KERNEL_AUTO, "tokens_on_n": M.MOE_FP8_KERNEL_TOKENS_ON_N,
                              "tokens_on_m": M.MOE_FP8_KERNEL_TOKENS_ON_M}[a.fp8_kernel])
-    FP8_FORM["value"] = a.fp8_kernel
     S = Setup(cfg, dev)
     T = cfg.T
     launches = M.moe_forward_launch_count(cfg, T)

@@ -392,6 +392,11 @@ enum {
 };
 MOE_API moe_status moe_select_fp8_kernel(int32_t which);
 
+/* The form moe_forward_fp8 runs for T tokens of this config under the current
+ * selection (AUTO resolved by the batch): MOE_FP8_KERNEL_TOKENS_ON_N or
+ * MOE_FP8_KERNEL_TOKENS_ON_M; -1 if the config or T is invalid. Host only. */
+MOE_API int32_t moe_fp8_kernel_for(const moe_config* cfg, int64_t T);
+
 /* Test hook for the failure path of the tensor-core pipelines, process-wide,
  * off by default; the pages have no counterpart. While enabled, one kernel
  * has its first CTA wait, before it issues anything, on a barrier phase that

@@ -43,7 +43,7 @@ EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_gate", "moe_dispatch
            "moe_stage_timing_begin_every", "moe_debug_stall_pipeline",
            "moe_gate_noalloc_check_error", "moe_experts_grouped_gather", "moe_forward_ep",
            "moe_cast_output", "moe_quantize_fp8", "moe_workspace_size_fp8", "moe_forward_fp8",
-           "moe_select_fp8_kernel")
+           "moe_select_fp8_kernel", "moe_fp8_kernel_for")
 
 # Kernels of moe_forward, in launch order.
 STAGES = ("router_logits", "router_select", "dispatch_rank", "dispatch_scan", "dispatch_pos",
@@ -90,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "moe_forward_launch_count": [C, I64],
         "moe_select_expert_kernel": [I32],
         "moe_select_fp8_kernel": [I32],
+        "moe_fp8_kernel_for": [C, I64],
         "moe_stage_timing_begin": [I32],
         "moe_stage_timing_begin_every": [I32, I32],
         "moe_debug_stall_pipeline": [I32],
@@ -284,6 +285,11 @@ def moe_select_expert_kernel(which: int) -> None:
 
 def moe_select_fp8_kernel(which: int) -> None:
     _check(_lib.moe_select_fp8_kernel(int(which)), "moe_select_fp8_kernel")
+
+
+def moe_fp8_kernel_for(cfg, T: int) -> int:
+    """The FP8 GEMM form moe_forward_fp8 runs for T tokens (MOE_FP8_KERNEL_TOKENS_ON_N / _ON_M)."""
+    return int(_lib.moe_fp8_kernel_for(_c(cfg), int(T)))
 
 
 def moe_stage_timing_begin(max_calls: int) -> None:

@@ -226,6 +226,13 @@ constexpr int64_t kGatherRows = 16;
 // the token-on-N form is faster below, the token-on-M form above).
 constexpr int64_t kFp8TokensOnMRows = 16;
 
+// Whether moe_forward_fp8 runs the token-on-M form for T tokens (the
+// selection, or AUTO's rule by the average rows per expert).
+bool fp8_tokens_on_m(const moe_config& c, int64_t T) {
+  return g_fp8_kernel == MOE_FP8_KERNEL_TOKENS_ON_M ||
+         (g_fp8_kernel == MOE_FP8_KERNEL_AUTO && T * (int64_t)c.topk > kFp8TokensOnMRows * c.n_routed);
+}
+
 bool fp8_shapes_ok(const moe_config& c) {
   const int B = kFp8Block;
   if (c.dtype != MOE_DT_BF16) return false;
@@ -585,9 +592,7 @@ moe_status moe_forward_fp8(const moe_config* cfg, int64_t T, const void* x, cons
   // x to e4m3 once per step, each block's scale also to the routed pairs'
   // permuted rows, and for the token-on-M form their codes too (its kernel
   // is timed with the up-projection)
-  const bool on_m = g_fp8_kernel == MOE_FP8_KERNEL_TOKENS_ON_M ||
-                    (g_fp8_kernel == MOE_FP8_KERNEL_AUTO &&
-                     T * (int64_t)c.topk > kFp8TokensOnMRows * c.n_routed);
+  const bool on_m = fp8_tokens_on_m(c, T);
   uint8_t* xq = at<uint8_t>(ws, F.xq);
   float* xs = at<float>(ws, F.xs);
   uint8_t* xq_perm = on_m ? at<uint8_t>(ws, F.xq_perm) : nullptr;
@@ -758,6 +763,11 @@ moe_status moe_select_expert_kernel(int32_t which) {
     return MOE_ERR_INVALID_ARG;
   g_expert_kernel = which;
   return MOE_OK;
+}
+
+int32_t moe_fp8_kernel_for(const moe_config* cfg, int64_t T) {
+  if (check_config(cfg, T) != MOE_OK) return -1;
+  return fp8_tokens_on_m(*cfg, T) ? MOE_FP8_KERNEL_TOKENS_ON_M : MOE_FP8_KERNEL_TOKENS_ON_N;
 }
 
 moe_status moe_select_fp8_kernel(int32_t which) {

@@ -95,6 +95,22 @@ def test_bad_sizes_and_pointers(M):
         assert M.raw_status("moe_select_fp8_kernel", which) == 0
 
 
+def test_fp8_form_for_a_batch(M):
+    # AUTO: tokens on M above 16 rows per expert on average (T * k > 16 * E)
+    from mixture_experts_layer_42_b200 import inputs
+    cfg = inputs.CONFIGS["v3_decode_fp8"]                   # k = 8, E = 256: T = 512 is 16 rows
+    assert M.moe_fp8_kernel_for(cfg, 512) == M.MOE_FP8_KERNEL_TOKENS_ON_N
+    assert M.moe_fp8_kernel_for(cfg, 513) == M.MOE_FP8_KERNEL_TOKENS_ON_M
+    assert M.moe_fp8_kernel_for(cfg, 0) == -1
+    try:
+        M.moe_select_fp8_kernel(M.MOE_FP8_KERNEL_TOKENS_ON_M)
+        assert M.moe_fp8_kernel_for(cfg, 1) == M.MOE_FP8_KERNEL_TOKENS_ON_M
+        M.moe_select_fp8_kernel(M.MOE_FP8_KERNEL_TOKENS_ON_N)
+        assert M.moe_fp8_kernel_for(cfg, 8192) == M.MOE_FP8_KERNEL_TOKENS_ON_N
+    finally:
+        M.moe_select_fp8_kernel(M.MOE_FP8_KERNEL_AUTO)
+
+
 def test_workspace_too_small_is_rejected_before_launch(M):
     n = ctypes.c_size_t(0)
     c = ctypes.byref(_cfg())
